@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Prefill throughput of the token-level sparse attention path on B200.
+
+One step = one prefill of the workload through the C ABI: the full-attention
+layer with selection (hs2_full_attn_select) followed by every sparse layer
+(hs2_sparse_attn), on inputs already resident in HBM.  The default workload is
+L = 131072 tokens, 64 query / 8 KV heads, head dim 128, full layer + 3 sparse
+layers (its Q/K/V/O tensors are far larger than the 126 MB L2, so no flush is
+needed between steps).
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl cuda|reference]
+
+Under torchrun every rank runs its own independent sequence (weak scaling,
+no collective on the data path); the step time is the max over ranks.
+`--impl reference` times the fp64 CPU oracle on a bounded sample instead.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "prefill tok/s (full-attn+select+sparse-attn) at 128k on 1 B200; % of roofline"
+
+
+# ------------------------------------------------------------ accounting --
+
+def algorithmic_work(wl) -> dict:
+    """Exact causal counts of what the method must compute or move."""
+    L, Hq, Hkv, d, B, k, w = wl.L, wl.Hq, wl.Hkv, wl.d, wl.block, wl.topk, wl.recent
+    fa = Hq * 4.0 * d * L * (L + 1) / 2
+    nb = L // B
+    e = np.minimum(L, B * (np.arange(nb) + 1)).astype(np.float64)
+    nc = np.maximum(0.0, e - w)
+    imp = Hq * 2.0 * d * B * nc.sum()
+    sel_rows = nc > k
+    select_bytes = Hkv * 4.0 * nc[sel_rows].sum()
+    glob = np.minimum(nc, k)
+    rec = np.minimum(w, e)
+    # visible pairs per block: every query sees the global part; query i sees
+    # recent positions [e_b - rec, i]
+    vis = B * glob + B * (B + 1) / 2.0 + B * (rec - B)   # rec >= B since recent >= block
+    sparse = Hq * 4.0 * d * vis.sum()
+    gather = Hkv * (glob + rec).sum() * 2 * 256.0
+    qo = 2.0 * L * Hq * d * 2
+    return {"fa_flop": fa, "imp_flop": imp, "select_bytes": select_bytes, "sparse_flop": sparse,
+            "gather_bytes": gather, "sparse_qo_bytes": qo}
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        self.dev = device_index
+
+    def __enter__(self):
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            target = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", target, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------ oracle baseline --
+
+class _Rows:
+    """Rows [s, e) of a [L][H][d] array addressed by absolute row index, so the
+    oracle can run one query block of a long sequence."""
+
+    def __init__(self, data, s, L):
+        self.data, self.s, self.shape = data, s, (L,) + data.shape[1:]
+
+    def __getitem__(self, key):
+        r, rest = key[0], tuple(key[1:])
+        if r == slice(None):
+            return _Rows(self.data[(slice(None),) + rest], self.s, self.shape[0])
+        return self.data[(slice(r.start - self.s, r.stop - self.s),) + rest]
+
+
+def _unit_flop(wl, b) -> float:
+    d, G, B = wl.d, wl.G, wl.block
+    e_b = min(wl.L, B * (b + 1))
+    n_c = max(0, e_b - wl.recent)
+    lst = min(n_c, wl.topk) + min(wl.recent, e_b)
+    return G * (4.0 * d * B * e_b + 2.0 * d * B * n_c + wl.n_sparse * 4.0 * d * B * lst)
+
+
+def oracle_units(wl, x, units):
+    """Run the fp64 oracle over (block, KV head) units of the workload whose
+    tensors live in `x` (torch, any device); returns elapsed seconds."""
+    from oracle import hs2_oracle as orc
+    from token_level_sparse_causal_b200 import inputs
+    G = wl.G
+    t = 0.0
+    for b, g in units:
+        s_b, e_b = b * wl.block, min(wl.L, (b + 1) * wl.block)
+        hs = slice(g * G, (g + 1) * G)
+        Qs = [_Rows(orc.decode_bf16(inputs.as_u16(q[s_b:e_b, hs])), s_b, wl.L) for q in x["q_layers"]]
+        K = orc.decode_bf16(inputs.as_u16(x["k"][:e_b, g:g + 1]))
+        V = orc.decode_bf16(inputs.as_u16(x["v"][:e_b, g:g + 1]))
+        t0 = time.perf_counter()
+        O, lse = orc.dense_attn(Qs[0], K, V, s_b, e_b)
+        I = orc.importance(Qs[0], K, lse, b, 0, wl.block, wl.recent)
+        idx, cnt = orc.select(I, wl.topk, wl.recent, e_b)
+        for Ql in Qs[1:]:
+            orc.sparse_attn(Ql, K, V, idx, cnt, b, 0, wl.block)
+        t += time.perf_counter() - t0
+    return t
+
+
+def sample_units(wl, seconds_target: float, rng_seed: int = 0, per_unit_s: float | None = None):
+    rng = np.random.default_rng(rng_seed)
+    first = max(0, -(-(wl.topk + wl.recent) // wl.block))
+    units = [(wl.nb - 1, 0)]
+    est_rate = 2.0e10  # fp64 flop/s guess, refined by the caller
+    budget = seconds_target * est_rate
+    used = _unit_flop(wl, wl.nb - 1)
+    while used < budget and len(units) < 64:
+        b = int(rng.integers(first, wl.nb))
+        g = int(rng.integers(0, wl.Hkv))
+        units.append((b, g))
+        used += _unit_flop(wl, b)
+    return units
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(wl, x, seconds_target: float) -> dict:
+    work = algorithmic_work(wl)
+    total = work["fa_flop"] + work["imp_flop"] + wl.n_sparse * work["sparse_flop"]
+    units = sample_units(wl, seconds_target)
+    t = oracle_units(wl, x, units)
+    sample = sum(_unit_flop(wl, b) for b, _ in units)
+    t_full = t * total / sample
+    return {"value": wl.L / t_full, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{len(units)} (query block, KV head) units of the {wl.name} workload "
+                      f"({t:.1f} s of fp64 NumPy), extrapolated to the whole prefill by the exact FLOP ratio"}
+
+
+# ------------------------------------------------------------- cuda arm --
+
+def run_cuda(args, wl, rank, world, dist):
+    import torch
+    from token_level_sparse_causal_b200 import build, hs2, inputs
+
+    build.build()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    my = wl.scaled(seed=wl.seed + 101 * rank) if world > 1 else wl
+    x = inputs.make_inputs(my, device=dev, with_needles=bool(my.needles))
+    q0, k, v = x["q_layers"][0], x["k"], x["v"]
+    shape = hs2.make_shape(q0, k, wl.topk, wl.recent)
+    out = hs2.alloc_outputs(shape, q0)
+    o_sp = [torch.empty_like(q) for q in x["q_layers"][1:]]
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hs2.hs2_full_attn_select(shape, q0, k, v, None, None, out["o"], out["lse"], out["idx"], out["cnt"],
+                                 out["workspace"], stream)
+        for ql, ol in zip(x["q_layers"][1:], o_sp):
+            hs2.hs2_sparse_attn(shape, ql, k, v, None, None, out["idx"], out["cnt"], ol, stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    hs2.hs2_sync(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    n0 = hs2.hs2_launch_count()
+    with ClockSampler(dev.index) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    launches = hs2.hs2_launch_count() - n0
+    hs2.hs2_sync(stream)
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / args.steps
+
+    # ---- per-stage device times (same stream, CUDA events), full kernel (1)
+    def timed(fn, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    n_stage = max(2, min(args.steps, 5))
+    fa_ms = timed(lambda: hs2.hs2_attn_fwd(shape, q0, k, v, None, None, out["o"], out["lse"], stream), n_stage)
+    sp_ms = timed(lambda: hs2.hs2_sparse_attn(shape, x["q_layers"][1], k, v, None, None, out["idx"], out["cnt"],
+                                              o_sp[0], stream), n_stage) if o_sp else 0.0
+    fs_ms = timed(lambda: hs2.hs2_full_attn_select(shape, q0, k, v, None, None, out["o"], out["lse"], out["idx"],
+                                                   out["cnt"], out["workspace"], stream), n_stage)
+    hs2.hs2_sync(stream)
+
+    # ---- end to end from pinned host buffers through the same C ABI calls
+    e2e = None
+    if not args.no_e2e:
+        h_in = [t.cpu().pin_memory() for t in x["q_layers"] + [k, v]]
+        d_in = [torch.empty_like(t) for t in x["q_layers"] + [k, v]]
+        outs = [out["o"]] + o_sp + [out["idx"], out["cnt"]]
+        h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        dq0, dk, dv = d_in[0], d_in[-2], d_in[-1]
+
+        def e2e_step():
+            for hsrc, ddst in zip(h_in, d_in):
+                ddst.copy_(hsrc, non_blocking=True)
+            hs2.hs2_full_attn_select(shape, dq0, dk, dv, None, None, out["o"], out["lse"], out["idx"], out["cnt"],
+                                     out["workspace"], stream)
+            for ql, ol in zip(d_in[1:-2], o_sp):
+                hs2.hs2_sparse_attn(shape, ql, dk, dv, None, None, out["idx"], out["cnt"], ol, stream)
+            for dsrc, hdst in zip(outs, h_out):
+                hdst.copy_(dsrc, non_blocking=True)
+
+        n_e2e = max(1, min(args.steps, 3))
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / n_e2e
+        if dist is not None:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        hs2.hs2_sync(stream)
+        e2e = {"value": world * wl.L / (e_ms / 1e3), "unit": "tok/s",
+               "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in h_in)),
+               "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in h_out)), "ms_per_step": e_ms}
+        del h_in, h_out, d_in
+
+    work = algorithmic_work(wl)
+    peaks = measured_peaks()
+    fa_tflops = work["fa_flop"] / (fa_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    res = {
+        "metric": METRIC, "value": world * wl.L / (ms / 1e3), "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "p50_ms": float(np.percentile(per, 50)), "p99_ms": float(np.percentile(per, 99)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; K from a 64-component Gaussian mixture, std 0.3)",
+        "config": {"workload": wl.name, "L": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
+                   "layers": f"1 full + {wl.n_sparse} sparse", "topk": wl.topk, "recent": wl.recent,
+                   "block": wl.block, "batch_per_gpu": 1, "parallelism": f"independent sequence per GPU x{world}",
+                   "l2": "inputs larger than L2 (Q alone is %.1f GB); no flush" % (q0.numel() * 2 / 1e9)},
+        "roofline": {"kernel": "fa_fwd (kernel 1, dense causal attention + LSE)", "bound": "tensor",
+                     "achieved": fa_tflops, "peak": peak, "unit": "TFLOP/s", "frac": fa_tflops / peak,
+                     "traffic": None,
+                     "peak_note": f"{peaks['source']} sustained bf16 (the kernel runs ~{fa_ms:.0f} ms per launch)"},
+        "stages_ms": {"fa_fwd": fa_ms, "importance+select": fs_ms - fa_ms, "sparse_attn_per_layer": sp_ms,
+                      "full_attn_select": fs_ms},
+        "stage_roofline": {
+            "fa_fwd_tflops": fa_tflops,
+            "importance_select_tflops": work["imp_flop"] / ((fs_ms - fa_ms) / 1e3) / 1e12 if fs_ms > fa_ms else None,
+            "sparse_tflops": work["sparse_flop"] / (sp_ms / 1e3) / 1e12 if sp_ms else None,
+            "sparse_gather_gbs": (work["gather_bytes"] + work["sparse_qo_bytes"]) / (sp_ms / 1e3) / 1e9 if sp_ms else None,
+            "path_roofline_ms": 1e3 * ((work["fa_flop"] + work["imp_flop"] + wl.n_sparse * work["sparse_flop"]) /
+                                       (peaks["bf16_tflops_sustained"] * 1e12) +
+                                       2 * work["select_bytes"] / (peaks["hbm_gbs"] * 1e9)),
+        },
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    res["stage_roofline"]["path_frac"] = res["stage_roofline"]["path_roofline_ms"] / ms
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl, x, args.cpu_seconds)
+    return res
+
+
+def run_reference(args, wl, rank, world):
+    """The fp64 oracle on the host cores, each step a bounded sample."""
+    import torch
+    from token_level_sparse_causal_b200 import inputs
+    if rank != 0:
+        return None
+    x = inputs.make_inputs(wl, device="cuda" if torch.cuda.is_available() else "cpu",
+                           with_needles=bool(wl.needles))
+    work = algorithmic_work(wl)
+    total = work["fa_flop"] + work["imp_flop"] + wl.n_sparse * work["sparse_flop"]
+    vals = []
+    for i in range(args.warmup + args.steps):
+        units = sample_units(wl, args.cpu_seconds / 3, rng_seed=i)
+        t = oracle_units(wl, x, units)
+        if i >= args.warmup:
+            vals.append(wl.L / (t * total / sum(_unit_flop(wl, b) for b, _ in units)))
+    v = float(np.median(vals))
+    return {"metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * wl.L / v, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "L": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
+                       "layers": f"1 full + {wl.n_sparse} sparse"},
+            "cpu_baseline": {"value": v, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": "per step: seeded (query block, KV head) units, extrapolated by FLOP ratio"},
+            "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--workload", default="c3", help="c1..c5 (default c3, the 128k workload)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample size for cpu_baseline")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "cuda":
+        ap.error("--warmup must be >= 3")
+
+    from token_level_sparse_causal_b200 import inputs
+    wl = inputs.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        if args.impl == "cuda":
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+            tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+            dist = tdist
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, wl, rank, world)
+        else:
+            res = run_cuda(args, wl, rank, world, dist)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,168 @@
+/*
+ * hs2.h -- C ABI of libhs2: token-level sparse causal attention for
+ * long-context prefill on one NVIDIA B200 (sm_100a).
+ *
+ * The method (HySparse2 architecture summary, "罗福莉剧透小米MiMo-V3架构：
+ * HySparse2让预填充提前退出"):
+ *   - a full-attention layer computes causal grouped-query attention and, from
+ *     its own complete scores, picks the tokens worth attending to
+ *     (ablation paragraph);
+ *   - selection is per token: the 1024 most important earlier tokens plus the
+ *     128 most recent ones (token-selection paragraph), the recent tokens
+ *     replacing the removed sliding-window branch (branch-removal paragraph);
+ *   - the following sparse layers reuse the full layer's KV cache and the
+ *     selected positions (KV-sharing paragraph, "KV Reuse").
+ * The attention itself is softmax(Q K^T / sqrt(d)) V (SHARP walk-through page,
+ * section 1.1) with the causal mask j <= i.
+ *
+ * Readings fixed by this library where the pages are silent:
+ *   - query head h uses KV head floor(h / G), G = Hq / Hkv;
+ *   - one index list per (query block of 64 tokens, KV head);
+ *   - importance of key j for block b, KV head g:
+ *       I_j = sum over the group's heads h and the block's queries i of
+ *             exp(s_hij - lse_hi),  s = q.k / sqrt(d), lse = natural-log LSE;
+ *   - candidates C_b = [0, e_b - recent), e_b = end of block b; the recent
+ *     window R_b = [e_b - recent, e_b) is always listed; ties in importance go
+ *     to the lower position; the list is ascending, -1 padded.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library allocates no device memory; calls are asynchronous on `stream`
+ *     (a cudaStream_t; NULL = the legacy default stream).  Only hs2_sync
+ *     blocks the host.
+ *   - Layouts are token-major, batch 1:
+ *       Q, O      : bf16 [L][Hq][d]     strides q_tok_stride / q_head_stride
+ *                                         (elements; O uses the same strides)
+ *       K, V      : bf16 or e4m3 [L][Hkv][d]   strides kv_tok_stride /
+ *                                         kv_head_stride (elements); the last
+ *                                         dimension is contiguous
+ *       k/v_scale : fp32 [L][Hkv] contiguous (only for kv_dtype = E4M3:
+ *                   stored value = e4m3(code) * scale)
+ *       lse       : fp32 [Hq][L]  (natural log)
+ *       idx       : int32 [Hkv][nb][topk + recent], nb = L / block,
+ *                   ascending positions, -1 padded
+ *       cnt       : int32 [Hkv][nb], valid entries per list
+ *   - Errors are returned as HS2_* codes; nothing is launched when an argument
+ *     check fails.  Faults found on the device (a bounded wait that ran out,
+ *     an index out of range) are recorded in a device status word and
+ *     returned by the next hs2_sync.
+ *   - Supported shapes: d = 128, block = 64, L a multiple of 64, recent a
+ *     multiple of 64 with recent >= block, 1 <= topk <= 4096 - recent,
+ *     G = Hq / Hkv in {2, 4, 8}, base pointers 16-byte aligned, strides
+ *     multiples of 8 elements (16 bytes for the byte-wide e4m3 cache: 16
+ *     elements).  Anything else returns HS2_ERR_UNSUPPORTED.
+ */
+#ifndef HS2_H_
+#define HS2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum hs2_status {
+  HS2_OK = 0,
+  HS2_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent shape */
+  HS2_ERR_UNSUPPORTED = 2,  /* shape/alignment outside the supported set above */
+  HS2_ERR_WORKSPACE = 3,    /* workspace smaller than the minimum */
+  HS2_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  HS2_ERR_TIMEOUT = 5,      /* a device-side bounded wait ran out */
+  HS2_ERR_INDEX = 6         /* an index list held a position outside [0, e_b) */
+};
+
+enum hs2_kv_dtype { HS2_KV_BF16 = 0, HS2_KV_E4M3 = 1 };
+
+typedef struct hs2_shape {
+  int32_t L, Hq, Hkv, d, block, topk, recent, kv_dtype;
+  int64_t q_tok_stride, q_head_stride;   /* elements of Q and O */
+  int64_t kv_tok_stride, kv_head_stride; /* elements of K and V */
+} hs2_shape;
+
+/*
+ * Full-attention layer + selection (the whole first half of the prefill path).
+ * Computes O and lse (causal GQA flash attention on tcgen05 tensor cores),
+ * then, in strips of query blocks that fit the workspace, the importance rows
+ * and their top-k selection, writing idx and cnt for every (KV head, block).
+ *
+ * workspace / workspace_bytes: scratch device memory for importance strips.
+ *   workspace == NULL: *workspace_bytes receives the recommended size (whole
+ *   path in as few strips as possible, capped so a strip stays L2-resident)
+ *   and nothing else happens.  Otherwise *workspace_bytes is the size of
+ *   `workspace` (16-byte aligned); it must be at least
+ *   Hkv * roundup(L - recent, 64) * 4 bytes (one block per strip), else
+ *   HS2_ERR_WORKSPACE.  The workspace holds no state between calls.
+ */
+int hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, const void* v,
+                         const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,
+                         int32_t* cnt, void* workspace, size_t* workspace_bytes, void* stream);
+
+/*
+ * One sparse layer (KV Reuse): for every query i of block b and head h,
+ * softmax over the listed positions j <= i of q_hi . k_j / sqrt(d), times V,
+ * using the shared K/V and the index lists written by hs2_full_attn_select.
+ * q is this layer's own Q; o (same layout and strides as q) is written.
+ * Padding entries (-1) are never dereferenced.
+ */
+int hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const void* v,
+                    const float* k_scale, const float* v_scale, const int32_t* idx, const int32_t* cnt,
+                    void* o, void* stream);
+
+/*
+ * Blocks until `stream` is idle, then returns the first error recorded on the
+ * device since the previous hs2_sync (and clears it), or HS2_ERR_CUDA if the
+ * stream reported an error, else HS2_OK.
+ */
+int hs2_sync(void* stream);
+
+/* ---- stage-level entry points (same kernels as above, one stage each) ---- */
+
+/* Full causal attention forward with LSE only (kernel 1 of the path). */
+int hs2_attn_fwd(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
+                 const float* v_scale, void* o, float* lse, void* stream);
+
+/*
+ * Importance rows (kernel 2) for query blocks [b0, b1), given the full
+ * layer's lse.  Row (g, b) holds I_j for j in C_b = [0, e_b - recent) at
+ * imp[((g * (b1 - b0)) + (b - b0)) * row_stride + j]; entries past |C_b| are
+ * not written.  row_stride (floats) must be a multiple of 4 and at least
+ * |C_{b1-1}|.
+ */
+int hs2_importance(const hs2_shape* shape, const void* q, const void* k, const float* k_scale,
+                   const float* lse, int32_t b0, int32_t b1, float* imp, int64_t row_stride, void* stream);
+
+/*
+ * Top-k + recent-window selection (kernel 3) over caller-supplied importance
+ * rows laid out as in hs2_importance, for blocks [b0, b1); writes the lists
+ * of those blocks into idx / cnt (full [Hkv][nb] layout).  Rows must hold
+ * finite values; -0.0 and +0.0 compare equal.
+ */
+int hs2_topk_select(const hs2_shape* shape, const float* imp, int64_t row_stride, int32_t b0, int32_t b1,
+                    int32_t* idx, int32_t* cnt, void* stream);
+
+/* ---- diagnostics ---- */
+
+/* Short text for an hs2_status code (static storage). */
+const char* hs2_strerror(int code);
+
+/*
+ * Limit for every device-side wait, in nanoseconds (default 2e9).  Test hook
+ * flags: bit 0 makes the attention kernels' load role issue nothing, so the
+ * bounded waits of the other roles must run out and hs2_sync must report
+ * HS2_ERR_TIMEOUT.  Flags are 0 in normal use.
+ */
+int hs2_debug_set(uint64_t wait_limit_ns, uint32_t flags);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int hs2_version(void);
+
+/* Number of kernels this library has launched since it was loaded (host-side
+ * counter, incremented once per successful launch; for accounting). */
+uint64_t hs2_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HS2_H_ */

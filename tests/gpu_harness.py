@@ -1,0 +1,96 @@
+"""Shared helpers for the GPU parity tests: run the CUDA path through the C ABI
+on seeded inputs, and hand the same input bytes to the fp64 oracle."""
+import numpy as np
+import torch
+
+from oracle import hs2_oracle as orc
+from token_level_sparse_causal_b200 import build, hs2, inputs
+
+# Tolerances: bf16 attention outputs max|d| <= 1.5e-2 and mean|d| <= 2e-3;
+# importance rtol 1e-3 (fp32); LSE is fp32 of a log-sum over <= 1M terms,
+# abs 2e-3 covers the fp32 accumulation of the row sum.
+O_MAX, O_MEAN, IMP_RTOL, LSE_ATOL = 1.5e-2, 2e-3, 1e-3, 2e-3
+GUARD = 4096
+WAIT_LIMIT_NS = 500_000_000   # every legitimate device wait here is far shorter
+SENTINEL_F = -12345.0
+
+
+def ensure_built():
+    build.build()
+    hs2.lib()
+
+
+def guarded(shape, dtype, device, fill=0):
+    """A tensor with guard bands of sentinels on both sides; returns (view, base)."""
+    n = int(np.prod(shape))
+    base = torch.full((n + 2 * GUARD,), SENTINEL_F if dtype.is_floating_point else -777, dtype=dtype, device=device)
+    view = base[GUARD:GUARD + n].view(*shape)
+    view.fill_(fill)
+    return view, base
+
+
+def guards_intact(base):
+    s = SENTINEL_F if base.dtype.is_floating_point else -777
+    return bool((base[:GUARD] == s).all() and (base[-GUARD:] == s).all())
+
+
+def decode(x):
+    """fp64 oracle inputs from the exact bytes the GPU reads."""
+    out = {"Q": [orc.decode_bf16(inputs.as_u16(q)) for q in x["q_layers"]]}
+    out["K"] = orc.decode_bf16(inputs.as_u16(x["k"]))
+    out["V"] = orc.decode_bf16(inputs.as_u16(x["v"]))
+    return out
+
+
+def to_dev(x, dev):
+    return {"q_layers": [q.to(dev) for q in x["q_layers"]], "k": x["k"].to(dev), "v": x["v"].to(dev)}
+
+
+def run_path(wl, xd, stream=None, guards=False):
+    """Full layer + every sparse layer through the C ABI; returns tensors."""
+    q0, k, v = xd["q_layers"][0], xd["k"], xd["v"]
+    dev = q0.device
+    shape = hs2.make_shape(q0, k, wl.topk, wl.recent)
+    nb = wl.L // wl.block
+    res = {"shape": shape, "bases": []}
+    if guards:
+        o, ob = guarded(q0.shape, torch.bfloat16, dev)
+        lse, lb = guarded((wl.Hq, wl.L), torch.float32, dev)
+        idx, ib = guarded((wl.Hkv, nb, wl.topk + wl.recent), torch.int32, dev)
+        cnt, cb = guarded((wl.Hkv, nb), torch.int32, dev)
+        res["bases"] += [ob, lb, ib, cb]
+    else:
+        o, lse = torch.empty_like(q0), torch.empty((wl.Hq, wl.L), device=dev, dtype=torch.float32)
+        idx = torch.empty((wl.Hkv, nb, wl.topk + wl.recent), device=dev, dtype=torch.int32)
+        cnt = torch.empty((wl.Hkv, nb), device=dev, dtype=torch.int32)
+    ws = torch.empty(hs2.workspace_bytes(shape) // 4 + 4, device=dev, dtype=torch.float32)
+    hs2.hs2_full_attn_select(shape, q0, k, v, None, None, o, lse, idx, cnt, ws, stream)
+    sparse = []
+    for ql in xd["q_layers"][1:]:
+        if guards:
+            ol, olb = guarded(ql.shape, torch.bfloat16, dev)
+            res["bases"].append(olb)
+        else:
+            ol = torch.empty_like(ql)
+        hs2.hs2_sparse_attn(shape, ql, k, v, None, None, idx, cnt, ol, stream)
+        sparse.append(ol)
+    hs2.hs2_sync(stream)
+    res.update(o=o, lse=lse, idx=idx, cnt=cnt, sparse=sparse)
+    return res
+
+
+def gpu_importance(shape, xd, lse, b0, b1):
+    """Exported fp32 importance rows for blocks [b0, b1) (kernel 2 alone)."""
+    L, recent = shape.L, shape.recent
+    stride = max(4, ((max(0, min(L, 64 * b1) - recent) + 3) // 4) * 4)
+    imp = torch.full((shape.Hkv, b1 - b0, stride), float("nan"), device=lse.device, dtype=torch.float32)
+    hs2.hs2_importance(shape, xd["q_layers"][0], xd["k"], None, lse, b0, b1, imp, stride)
+    hs2.hs2_sync()
+    return imp
+
+
+def bf16_close(got, ref, what=""):
+    d = np.abs(np.asarray(got, dtype=np.float64) - ref)
+    assert d.max() <= O_MAX, f"{what}: max|d| {d.max():.3e} > {O_MAX}"
+    assert d.mean() <= O_MEAN, f"{what}: mean|d| {d.mean():.3e} > {O_MEAN}"
+    return d.max(), d.mean()

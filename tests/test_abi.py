@@ -1,0 +1,143 @@
+"""The C ABI without a GPU: libhs2.so loads, exports every function that
+include/hs2.h declares, answers the workspace query, and rejects bad
+arguments with the documented codes before touching the device.
+
+Every call below that passes pointers is built to fail a host-side check
+(the fake addresses are never dereferenced or launched on)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from token_level_sparse_causal_b200 import build, hs2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return hs2.lib()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "hs2.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hs2_[a-z_0-9]+)\s*\(", text)))
+
+
+def _shape(**kw):
+    base = dict(L=2048, Hq=8, Hkv=2, d=128, block=64, topk=1024, recent=128, kv_dtype=0,
+                q_tok_stride=8 * 128, q_head_stride=128, kv_tok_stride=2 * 128, kv_head_stride=128)
+    base.update(kw)
+    return hs2.Hs2Shape(**base)
+
+
+P = ctypes.c_void_p(0x10000)        # aligned fake address, never dereferenced
+MIS = ctypes.c_void_p(0x10008)      # misaligned fake address
+
+
+def test_exports_match_header(lib):
+    names = _declared()
+    assert set(names) == set(hs2.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", hs2.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (hs2_[a-z_0-9]+)", out))
+    assert set(names) <= exported
+    assert not [s for s in exported if not s.startswith("hs2_")], "only hs2_* symbols are exported"
+
+
+def test_no_link_time_driver_dependency():
+    out = subprocess.run(["ldd", hs2.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libtorch" not in out
+
+
+def test_strerror_and_version(lib):
+    assert hs2.strerror(0) == "ok"
+    assert "timed out" in hs2.strerror(hs2.HS2_ERR_TIMEOUT)
+    assert hs2.strerror(999).startswith("unknown")
+    assert lib.hs2_version() >= 100
+
+
+def test_workspace_query_is_host_only(lib):
+    s = _shape(L=131072, Hq=64, Hkv=8, q_tok_stride=64 * 128, kv_tok_stride=8 * 128)
+    n = hs2.workspace_bytes(s)
+    min_ws = 8 * (131072 - 128) * 4
+    assert min_ws <= n <= max(min_ws, 64 << 20)
+    small = _shape(L=1024)
+    assert hs2.workspace_bytes(small) >= 2 * (1024 - 128) * 4
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=64), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(block=32), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(L=2000), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(L=0), hs2.HS2_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), hs2.HS2_ERR_INVALID_ARG),
+    (dict(Hq=16, Hkv=1, q_tok_stride=16 * 128, kv_tok_stride=128), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(Hq=2, Hkv=2, q_tok_stride=2 * 128), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(recent=32), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(recent=100), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(topk=4000), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(kv_dtype=7), hs2.HS2_ERR_INVALID_ARG),
+    (dict(q_tok_stride=8 * 128 + 4), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(q_tok_stride=4 * 128), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(kv_head_stride=64), hs2.HS2_ERR_UNSUPPORTED),
+])
+def test_bad_shapes_rejected(lib, kw, code):
+    s = ctypes.byref(_shape(**kw))
+    st = ctypes.c_void_p(0)
+    assert lib.hs2_attn_fwd(s, P, P, P, None, None, P, P, st) == code
+    assert lib.hs2_sparse_attn(s, P, P, P, None, None, P, P, P, st) == code
+    n = ctypes.c_size_t(1 << 30)
+    assert lib.hs2_full_attn_select(s, P, P, P, None, None, P, P, P, P, P, ctypes.byref(n), st) == code
+    assert lib.hs2_importance(s, P, P, None, P, 0, 1, P, 4096, st) == code
+    assert lib.hs2_topk_select(s, P, 4096, 0, 1, P, P, st) == code
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    s = ctypes.byref(_shape())
+    st = ctypes.c_void_p(0)
+    assert lib.hs2_attn_fwd(s, None, P, P, None, None, P, P, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_attn_fwd(s, P, None, P, None, None, P, P, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_attn_fwd(s, P, P, P, None, None, P, None, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_attn_fwd(s, MIS, P, P, None, None, P, P, st) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_attn_fwd(s, P, MIS, P, None, None, P, P, st) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_sparse_attn(s, P, P, P, None, None, None, P, P, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_sparse_attn(s, P, P, P, None, None, P, P, MIS, st) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_topk_select(s, None, 4096, 0, 1, P, P, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_topk_select(s, MIS, 4096, 0, 1, P, P, st) == hs2.HS2_ERR_UNSUPPORTED
+
+
+def test_block_ranges_and_strides_rejected(lib):
+    s = ctypes.byref(_shape())
+    st = ctypes.c_void_p(0)
+    assert lib.hs2_importance(s, P, P, None, P, 3, 3, P, 4096, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_importance(s, P, P, None, P, 0, 33, P, 4096, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_importance(s, P, P, None, P, 0, 32, P, 1900, st) == hs2.HS2_ERR_INVALID_ARG   # < |C_31|
+    assert lib.hs2_importance(s, P, P, None, P, 0, 32, P, 4098, st) == hs2.HS2_ERR_INVALID_ARG   # not % 4
+    assert lib.hs2_topk_select(s, P, 4096, -1, 4, P, P, st) == hs2.HS2_ERR_INVALID_ARG
+
+
+def test_workspace_too_small_rejected(lib):
+    s = _shape()
+    n = ctypes.c_size_t(2 * (2048 - 128) * 4 - 16)
+    rc = lib.hs2_full_attn_select(ctypes.byref(s), P, P, P, None, None, P, P, P, P, P, ctypes.byref(n),
+                                  ctypes.c_void_p(0))
+    assert rc == hs2.HS2_ERR_WORKSPACE
+    assert lib.hs2_full_attn_select(ctypes.byref(s), P, P, P, None, None, P, P, P, P, P, None,
+                                    ctypes.c_void_p(0)) == hs2.HS2_ERR_INVALID_ARG
+
+
+def test_fp8_needs_scales(lib):
+    s = ctypes.byref(_shape(kv_dtype=1))
+    st = ctypes.c_void_p(0)
+    assert lib.hs2_attn_fwd(s, P, P, P, None, None, P, P, st) in (hs2.HS2_ERR_INVALID_ARG, hs2.HS2_ERR_UNSUPPORTED)
+
+
+def test_debug_set_validates(lib):
+    assert lib.hs2_debug_set(0, 0) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_debug_set(2_000_000_000, 0) == hs2.HS2_OK

@@ -1,0 +1,346 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle on the same
+seeded input bytes.
+
+Bars: indices bit-exact when both sides select from the same exported fp32
+importance; importance within rtol 1e-3; bf16 attention outputs within
+max|d| <= 1.5e-2 and mean|d| <= 2e-3.  Small shapes are checked on every
+output element and span several tiles with ragged tails; the 32k and 128k
+workloads (the latter in the launch configuration the benchmark times) are
+checked on sampled query blocks."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import hs2_oracle as orc
+from tests import gpu_harness as H
+from token_level_sparse_causal_b200 import hs2, inputs
+
+pytestmark = pytest.mark.gpu
+
+DEV = torch.device("cuda:0")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    H.ensure_built()
+    hs2.hs2_debug_set(H.WAIT_LIMIT_NS, 0)
+
+
+def _wl(L, Hq, Hkv, n_sparse=1, seed=7, topk=1024, recent=128, needles=()):
+    return inputs.Workload(f"t{L}_{Hq}x{Hkv}", L, Hq, Hkv, n_sparse, seed, needles=needles, topk=topk, recent=recent)
+
+
+# ------------------------------------------------------------ kernel (1) --
+
+@pytest.mark.parametrize("L,Hq,Hkv", [(1088, 8, 4), (2048, 4, 1), (640, 16, 2)])
+def test_attn_fwd_matches_oracle(L, Hq, Hkv):
+    wl = _wl(L, Hq, Hkv)
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    shape = hs2.make_shape(xd["q_layers"][0], xd["k"])
+    o, ob = H.guarded((L, Hq, 128), torch.bfloat16, DEV)
+    lse, lb = H.guarded((Hq, L), torch.float32, DEV)
+    hs2.hs2_attn_fwd(shape, xd["q_layers"][0], xd["k"], xd["v"], None, None, o, lse)
+    hs2.hs2_sync()
+    D = H.decode(x)
+    O, LSE = orc.dense_attn(D["Q"][0], D["K"], D["V"])
+    H.bf16_close(o.float().cpu().numpy(), O, "O")
+    assert np.abs(lse.cpu().numpy() - LSE).max() <= H.LSE_ATOL
+    assert H.guards_intact(ob) and H.guards_intact(lb)
+
+
+def test_attn_fwd_on_a_side_stream_with_padded_strides():
+    """Non-default stream; Q/O with a padded head stride and K/V with a padded
+    token stride (strides are honoured, nothing outside the rows is read)."""
+    L, Hq, Hkv = 512, 8, 2
+    wl = _wl(L, Hq, Hkv, seed=3)
+    x = inputs.make_inputs(wl)
+    qpad = torch.zeros((L, Hq, 136), dtype=torch.bfloat16)
+    qpad[:, :, :128] = x["q_layers"][0]
+    kpad = torch.zeros((L, Hkv + 1, 128), dtype=torch.bfloat16)
+    vpad = torch.zeros((L, Hkv + 1, 128), dtype=torch.bfloat16)
+    kpad[:, :Hkv], vpad[:, :Hkv] = x["k"], x["v"]
+    q = qpad.to(DEV)[:, :, :128]
+    k, v = kpad.to(DEV)[:, :Hkv], vpad.to(DEV)[:, :Hkv]
+    shape = hs2.make_shape(q, k)
+    assert shape.q_head_stride == 136 and shape.kv_tok_stride == (Hkv + 1) * 128
+    o = torch.zeros((L, Hq, 136), dtype=torch.bfloat16, device=DEV)[:, :, :128]
+    lse = torch.empty((Hq, L), device=DEV)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        hs2.hs2_attn_fwd(shape, q, k, v, None, None, o, lse, stream=s)
+        hs2.hs2_sync(s)
+    D = H.decode(x)
+    O, LSE = orc.dense_attn(D["Q"][0], D["K"], D["V"])
+    H.bf16_close(o.float().cpu().numpy(), O, "O")
+    assert np.abs(lse.cpu().numpy() - LSE).max() <= H.LSE_ATOL
+
+
+# ------------------------------------------------------------ kernel (2) --
+
+@pytest.mark.parametrize("L,Hq,Hkv", [(2304, 8, 1), (1536, 8, 2), (1024, 4, 2)])
+def test_importance_matches_oracle(L, Hq, Hkv):
+    wl = _wl(L, Hq, Hkv, seed=11)
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    shape = hs2.make_shape(xd["q_layers"][0], xd["k"])
+    o = torch.empty_like(xd["q_layers"][0])
+    lse = torch.empty((Hq, L), device=DEV)
+    hs2.hs2_attn_fwd(shape, xd["q_layers"][0], xd["k"], xd["v"], None, None, o, lse)
+    nb = L // 64
+    imp = H.gpu_importance(shape, xd, lse, 0, nb).cpu().numpy()
+    D = H.decode(x)
+    _, LSE = orc.dense_attn(D["Q"][0], D["K"], D["V"])
+    worst = 0.0
+    for b in range(nb):
+        s_b, e_b = orc.block_rows(b, L, 64)
+        for g in range(Hkv):
+            ref = orc.importance(D["Q"][0], D["K"], LSE[:, s_b:e_b], b, g, 64, 128)
+            got = imp[g, b, :ref.size]
+            assert np.all(np.isfinite(got))
+            rel = np.abs(got - ref) / np.maximum(np.abs(ref), 1e-30)
+            worst = max(worst, rel.max() if ref.size else 0.0)
+    assert worst <= H.IMP_RTOL, worst
+
+
+# ------------------------------------------------------------ kernel (3) --
+
+@pytest.mark.parametrize("L,Hq,Hkv", [(2304, 8, 1), (1536, 8, 2)])
+def test_select_bit_exact_on_exported_importance(L, Hq, Hkv):
+    wl = _wl(L, Hq, Hkv, seed=13)
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    r = H.run_path(wl, xd, guards=True)
+    nb = L // 64
+    imp = H.gpu_importance(r["shape"], xd, r["lse"], 0, nb).cpu().numpy().astype(np.float64)
+    idx, cnt = r["idx"].cpu().numpy(), r["cnt"].cpu().numpy()
+    for b in range(nb):
+        _, e_b = orc.block_rows(b, L, 64)
+        n_c = orc.n_candidates(e_b, 128)
+        for g in range(Hkv):
+            want, wc = orc.select(imp[g, b, :n_c], 1024, 128, e_b)
+            assert cnt[g, b] == wc
+            assert np.array_equal(idx[g, b], want), (g, b)
+    assert all(H.guards_intact(bb) for bb in r["bases"])
+
+
+def _crafted_rows(n, rng):
+    kinds = [
+        rng.random(n).astype(np.float32),                                   # distinct
+        (rng.integers(0, 4, n) / 4.0).astype(np.float32),                   # 4 levels: huge ties
+        np.ones(n, np.float32),                                             # all equal
+        np.where(rng.random(n) < 0.5, -0.0, 0.0).astype(np.float32),        # +-0 only
+        np.exp(-rng.random(n) * 80).astype(np.float32),                     # wide dynamic range
+        np.concatenate([np.zeros(n - 1100, np.float32), np.full(1100, 1e-3, np.float32)]),  # tail-heavy
+    ]
+    return kinds
+
+
+def test_select_crafted_rows_bit_exact():
+    L, Hkv, topk, recent = 8192, 6, 1024, 128
+    shape = hs2.Hs2Shape(L=L, Hq=12, Hkv=Hkv, d=128, block=64, topk=topk, recent=recent, kv_dtype=0,
+                         q_tok_stride=12 * 128, q_head_stride=128, kv_tok_stride=Hkv * 128, kv_head_stride=128)
+    nb = L // 64
+    rng = np.random.default_rng(5)
+    for b0, b1 in [(0, 24), (100, 104), (nb - 3, nb)]:
+        stride = ((orc.n_candidates(64 * b1, recent) + 3) // 4) * 4
+        rows = np.full((Hkv, b1 - b0, max(stride, 4)), np.nan, np.float32)
+        for bi, b in enumerate(range(b0, b1)):
+            n_c = orc.n_candidates(64 * (b + 1), recent)
+            if n_c == 0:
+                continue
+            for g, row in enumerate(_crafted_rows(max(n_c, 1100), rng)):
+                rows[g, bi, :n_c] = row[:n_c]
+        imp = torch.from_numpy(rows).to(DEV)
+        idx = torch.full((Hkv, nb, topk + recent), -9, dtype=torch.int32, device=DEV)
+        cnt = torch.full((Hkv, nb), -9, dtype=torch.int32, device=DEV)
+        hs2.hs2_topk_select(shape, imp, rows.shape[2], b0, b1, idx, cnt)
+        hs2.hs2_sync()
+        idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+        for bi, b in enumerate(range(b0, b1)):
+            e_b = 64 * (b + 1)
+            n_c = orc.n_candidates(e_b, recent)
+            for g in range(Hkv):
+                want, wc = orc.select(rows[g, bi, :n_c].astype(np.float64), topk, recent, e_b)
+                assert cnt_h[g, b] == wc and np.array_equal(idx_h[g, b], want), (b, g)
+        untouched = [bb for bb in range(nb) if not b0 <= bb < b1]
+        assert np.all(idx_h[:, untouched] == -9) and np.all(cnt_h[:, untouched] == -9)
+
+
+# ------------------------------------------------------------ kernel (4) --
+
+def test_sparse_matches_oracle_on_gpu_lists():
+    L, Hq, Hkv = 4096, 8, 2
+    wl = _wl(L, Hq, Hkv, n_sparse=2, seed=17, topk=1000)          # 1128-entry lists: ragged last tile
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    r = H.run_path(wl, xd, guards=True)
+    D = H.decode(x)
+    idx, cnt = r["idx"].cpu().numpy(), r["cnt"].cpu().numpy()
+    G = wl.G
+    for layer, ol in enumerate(r["sparse"], start=1):
+        got = ol.float().cpu().numpy()
+        ref = np.empty_like(got, dtype=np.float64)
+        for b in range(L // 64):
+            s_b, e_b = orc.block_rows(b, L, 64)
+            for g in range(Hkv):
+                ref[s_b:e_b, g * G:(g + 1) * G] = orc.sparse_attn(D["Q"][layer], D["K"], D["V"], idx[g, b],
+                                                                  int(cnt[g, b]), b, g, 64)
+        H.bf16_close(got, ref, f"sparse layer {layer}")
+    assert all(H.guards_intact(bb) for bb in r["bases"])
+
+
+@pytest.mark.parametrize("L", [1152, 640])
+def test_sparse_equals_dense_when_lists_cover_everything(L):
+    wl = _wl(L, 8, 2, n_sparse=1, seed=19)
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    r = H.run_path(wl, xd)
+    cnt = r["cnt"].cpu().numpy()
+    assert np.array_equal(cnt, np.broadcast_to(np.arange(1, L // 64 + 1) * 64, cnt.shape))
+    D = H.decode(x)
+    O1, _ = orc.dense_attn(D["Q"][1], D["K"], D["V"])
+    H.bf16_close(r["sparse"][0].float().cpu().numpy(), O1, "sparse == dense")
+
+
+# ----------------------------------------------------------- whole path --
+
+def test_end_to_end_2k_workload_with_needles():
+    wl = inputs.WORKLOADS["c1"]
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    r = H.run_path(wl, xd, guards=True)
+    D = H.decode(x)
+    O, LSE = orc.dense_attn(D["Q"][0], D["K"], D["V"])
+    H.bf16_close(r["o"].float().cpu().numpy(), O, "full-layer O")
+    assert np.abs(r["lse"].cpu().numpy() - LSE).max() <= H.LSE_ATOL
+    nb = wl.L // 64
+    imp = H.gpu_importance(r["shape"], xd, r["lse"], 0, nb).cpu().numpy().astype(np.float64)
+    idx, cnt = r["idx"].cpu().numpy(), r["cnt"].cpu().numpy()
+    ref_sp = np.empty((wl.L, wl.Hq, 128))
+    for b in range(nb):
+        s_b, e_b = orc.block_rows(b, wl.L, 64)
+        want, wc = orc.select(imp[0, b, :orc.n_candidates(e_b, 128)], 1024, 128, e_b)
+        assert np.array_equal(idx[0, b], want) and cnt[0, b] == wc
+        ref_sp[s_b:e_b] = orc.sparse_attn(D["Q"][1], D["K"], D["V"], idx[0, b], wc, b, 0, 64)
+    H.bf16_close(r["sparse"][0].float().cpu().numpy(), ref_sp, "sparse layer")
+    hit = sum(int(n["p"] in set(idx[n["g"], n["t"] // 64, :cnt[n["g"], n["t"] // 64]].tolist()))
+              for n in x["needles"])
+    print(f"needle recall {hit}/{len(x['needles'])}")
+    assert all(H.guards_intact(bb) for bb in r["bases"])
+
+
+class _Rows:
+    """Rows [s, e) of a [L][H][d] array, addressed by absolute row index, so
+    the oracle can evaluate one query block of a long workload."""
+
+    def __init__(self, data, s, L):
+        self.data, self.s, self.shape = data, s, (L,) + data.shape[1:]
+
+    def __getitem__(self, key):
+        r, rest = key[0], tuple(key[1:])
+        if r == slice(None):
+            return _Rows(self.data[(slice(None),) + rest], self.s, self.shape[0])
+        assert r.start >= self.s
+        return self.data[(slice(r.start - self.s, r.stop - self.s),) + rest]
+
+
+def _sampled_check(wl, blocks, groups):
+    xd = inputs.make_inputs(wl, device=DEV)
+    r = H.run_path(wl, xd)
+    G = wl.G
+    for b in blocks:
+        s_b, e_b = orc.block_rows(b, wl.L, 64)
+        imp = H.gpu_importance(r["shape"], xd, r["lse"], b, b + 1).cpu().numpy().astype(np.float64)
+        for g in groups:
+            hs = slice(g * G, (g + 1) * G)
+            Qb = [_Rows(orc.decode_bf16(inputs.as_u16(q[s_b:e_b, hs])), s_b, wl.L) for q in xd["q_layers"]]
+            K = orc.decode_bf16(inputs.as_u16(xd["k"][:e_b, g:g + 1]))
+            V = orc.decode_bf16(inputs.as_u16(xd["v"][:e_b, g:g + 1]))
+            O, LSE = orc.dense_attn(Qb[0], K, V, s_b, e_b)
+            H.bf16_close(r["o"][s_b:e_b, hs].float().cpu().numpy(), O, f"O b{b} g{g}")
+            assert np.abs(r["lse"][hs, s_b:e_b].cpu().numpy() - LSE).max() <= H.LSE_ATOL
+            lse_full = np.zeros((G, e_b - s_b))
+            lse_full[:] = LSE
+            ref_imp = orc.importance(Qb[0], K, lse_full, b, 0, 64, wl.recent)
+            got_imp = imp[g, 0, :ref_imp.size]
+            rel = np.abs(got_imp - ref_imp) / np.maximum(np.abs(ref_imp), 1e-30)
+            assert rel.max() <= H.IMP_RTOL, (b, g, rel.max())
+            want, wc = orc.select(got_imp, wl.topk, wl.recent, e_b)
+            idx_g = r["idx"][g, b].cpu().numpy()
+            assert int(r["cnt"][g, b]) == wc and np.array_equal(idx_g, want), (b, g)
+            for layer, ol in enumerate(r["sparse"], start=1):
+                ref = orc.sparse_attn(Qb[layer], K, V, idx_g, wc, b, 0, 64)
+                H.bf16_close(ol[s_b:e_b, hs].float().cpu().numpy(), ref, f"sparse l{layer} b{b} g{g}")
+    return r
+
+
+def test_full_size_32k_workload_sampled():
+    wl = inputs.WORKLOADS["c2"]
+    rng = np.random.default_rng(1)
+    blocks = [18, wl.nb - 1] + [int(b) for b in rng.integers(19, wl.nb - 1, 2)]
+    _sampled_check(wl, blocks, groups=[0, 5])
+
+
+def test_full_size_128k_workload_sampled():
+    """The benchmark's workload and launch configuration."""
+    wl = inputs.WORKLOADS["c3"]
+    rng = np.random.default_rng(2)
+    blocks = [18, wl.nb - 1] + [int(b) for b in rng.integers(19, wl.nb - 1, 2)]
+    _sampled_check(wl, blocks, groups=[3, 7])
+    torch.cuda.empty_cache()
+
+
+# -------------------------------------------------- device-side failures --
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """The load role issues nothing (test flag), so the other roles' bounded
+    waits run out: hs2_sync reports HS2_ERR_TIMEOUT, and the next call works."""
+    wl = _wl(256, 4, 2, seed=23)
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    shape = hs2.make_shape(xd["q_layers"][0], xd["k"])
+    o = torch.empty_like(xd["q_layers"][0])
+    lse = torch.empty((4, 256), device=DEV)
+    hs2.hs2_debug_set(50_000_000, 1)
+    try:
+        hs2.hs2_attn_fwd(shape, xd["q_layers"][0], xd["k"], xd["v"], None, None, o, lse)
+        with pytest.raises(hs2.Hs2Error) as e:
+            hs2.hs2_sync()
+        assert e.value.code == hs2.HS2_ERR_TIMEOUT
+    finally:
+        hs2.hs2_debug_set(H.WAIT_LIMIT_NS, 0)
+    hs2.hs2_attn_fwd(shape, xd["q_layers"][0], xd["k"], xd["v"], None, None, o, lse)
+    hs2.hs2_sync()
+    D = H.decode(x)
+    O, _ = orc.dense_attn(D["Q"][0], D["K"], D["V"])
+    H.bf16_close(o.float().cpu().numpy(), O, "O after timeout")
+
+
+def test_out_of_range_list_entries_are_reported_not_read():
+    """Listed positions outside [0, e_b) are never dereferenced: the gather
+    zero-fills them, the softmax masks them, and hs2_sync reports
+    HS2_ERR_INDEX; the remaining entries give the right answer."""
+    L, Hq, Hkv = 512, 4, 2
+    wl = _wl(L, Hq, Hkv, seed=29)
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    r = H.run_path(wl, xd)
+    idx = r["idx"].clone()
+    b = 5
+    idx[1, b, 3] = 64 * (b + 1) + 7       # beyond the block end
+    idx[1, b, 10] = -5                    # negative
+    o = torch.empty_like(xd["q_layers"][1])
+    hs2.hs2_sparse_attn(r["shape"], xd["q_layers"][1], xd["k"], xd["v"], None, None, idx, r["cnt"], o)
+    with pytest.raises(hs2.Hs2Error) as e:
+        hs2.hs2_sync()
+    assert e.value.code == hs2.HS2_ERR_INDEX
+    D = H.decode(x)
+    lst = idx[1, b].cpu().numpy()
+    c = int(r["cnt"][1, b])
+    keep = lst[:c][(lst[:c] >= 0) & (lst[:c] < 64 * (b + 1))]
+    ref = orc.sparse_attn(D["Q"][1], D["K"], D["V"], keep, keep.size, b, 1, 64)
+    H.bf16_close(o[64 * b:64 * (b + 1), 2:4].float().cpu().numpy(), ref, "masked bad entries")
+    hs2.hs2_sync()   # status was cleared

@@ -1,0 +1,390 @@
+// libhs2: host side of the C ABI declared in include/hs2.h, plus the single
+// translation unit that instantiates every sm_100a kernel.
+//
+// Host responsibilities: argument validation (nothing is launched when a
+// check fails), TMA tensor-map encoding, the strip schedule of the importance
+// and select passes, launches on the caller's stream, and the device status
+// word read back by hs2_sync.  No device memory is ever allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/hs2.h"
+#include "common.cuh"
+#include "flash.cuh"
+#include "importance.cuh"
+#include "topk_select.cuh"
+
+namespace hs2 {
+namespace {
+
+uint64_t g_wait_limit_ns = 2000000000ull;
+uint32_t g_flags = 0;
+std::atomic<uint64_t> g_launches{0};
+
+inline int cuda_ok(cudaError_t e) { return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA; }
+
+inline int launched() {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return HS2_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return HS2_OK;
+}
+
+// ------------------------------------------------------------ validation --
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+int check_shape(const hs2_shape* s) {
+  if (!s) return HS2_ERR_INVALID_ARG;
+  if (s->L <= 0 || s->Hq <= 0 || s->Hkv <= 0 || s->d <= 0 || s->block <= 0 || s->topk <= 0 || s->recent <= 0)
+    return HS2_ERR_INVALID_ARG;
+  if (s->Hq % s->Hkv != 0) return HS2_ERR_INVALID_ARG;
+  if (s->kv_dtype != HS2_KV_BF16 && s->kv_dtype != HS2_KV_E4M3) return HS2_ERR_INVALID_ARG;
+  if (s->q_tok_stride <= 0 || s->q_head_stride <= 0 || s->kv_tok_stride <= 0 || s->kv_head_stride <= 0)
+    return HS2_ERR_INVALID_ARG;
+  const int G = s->Hq / s->Hkv;
+  if (s->d != HD || s->block != 64) return HS2_ERR_UNSUPPORTED;
+  if (s->L % 64 != 0 || s->L > (1 << 24)) return HS2_ERR_UNSUPPORTED;
+  if (s->recent % 64 != 0 || s->recent < s->block) return HS2_ERR_UNSUPPORTED;
+  if (s->topk + s->recent > MAX_LIST) return HS2_ERR_UNSUPPORTED;
+  if (G != 2 && G != 4 && G != 8) return HS2_ERR_UNSUPPORTED;
+  if (s->q_tok_stride % 8 || s->q_head_stride % 8) return HS2_ERR_UNSUPPORTED;
+  const int64_t kv_align = (s->kv_dtype == HS2_KV_E4M3) ? 16 : 8;
+  if (s->kv_tok_stride % kv_align || s->kv_head_stride % kv_align) return HS2_ERR_UNSUPPORTED;
+  // rows must not overlap: d contiguous elements per head, heads within a token
+  if (s->q_head_stride < HD || s->kv_head_stride < HD) return HS2_ERR_UNSUPPORTED;
+  if (s->q_tok_stride < static_cast<int64_t>(s->Hq) * s->q_head_stride) return HS2_ERR_UNSUPPORTED;
+  if (s->kv_tok_stride < static_cast<int64_t>(s->Hkv) * s->kv_head_stride) return HS2_ERR_UNSUPPORTED;
+  if (s->kv_dtype == HS2_KV_E4M3) return HS2_ERR_UNSUPPORTED;  // FP8 cache: not built yet
+  return HS2_OK;
+}
+
+int check_kv(const hs2_shape* s, const void* k, const void* v, const float* ks, const float* vs) {
+  if (!k || !v) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v)) return HS2_ERR_UNSUPPORTED;
+  if (s->kv_dtype == HS2_KV_E4M3 && (!ks || !vs)) return HS2_ERR_INVALID_ARG;
+  return HS2_OK;
+}
+
+// --------------------------------------------------------- tensor maps --
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 map over [tokens][heads][128] with the d dimension contiguous and
+// a box of (64 d, box_h heads, box_t tokens), 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* base, int L, int H, int64_t tok_stride, int64_t head_stride, int box_h,
+             int box_t) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return HS2_ERR_CUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(HD), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(L)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_stride) * 2, static_cast<cuuint64_t>(tok_stride) * 2};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_h), static_cast<cuuint32_t>(box_t)};
+  const cuuint32_t es[3] = {1u, 1u, 1u};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HS2_OK : HS2_ERR_CUDA;
+}
+
+float scale_log2(int d) { return static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d))); }
+
+template <typename K>
+int set_smem(K kernel, uint32_t bytes) {
+  return cuda_ok(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)));
+}
+
+// ------------------------------------------------------------- launches --
+
+int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void* v, void* o, float* lse,
+                    cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  int rc;
+  if ((rc = make_map(&mq, q, s->L, s->Hq, s->q_tok_stride, s->q_head_stride, 1, 128))) return rc;
+  if ((rc = make_map(&mk, k, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+  if ((rc = make_map(&mv, v, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+  FlashParams p{};
+  p.L = s->L;
+  p.Hq = s->Hq;
+  p.Hkv = s->Hkv;
+  p.G = s->Hq / s->Hkv;
+  p.nqt = s->L / 128 + (s->L % 128 ? 1 : 0);
+  p.scale_log2 = scale_log2(s->d);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_tok = s->q_tok_stride;
+  p.o_head = s->q_head_stride;
+  p.lse = lse;
+  p.limit_ns = g_wait_limit_ns;
+  p.flags = g_flags;
+  static int attr = set_smem(flash_fwd_kernel<FLASH_DENSE>, FL_SMEM_DENSE);
+  if (attr) return attr;
+  const unsigned grid = static_cast<unsigned>(p.nqt * s->Hq);
+  flash_fwd_kernel<FLASH_DENSE><<<grid, 256, FL_SMEM_DENSE, st>>>(mq, mk, mv, p);
+  return launched();
+}
+
+int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* v, const int32_t* idx,
+                  const int32_t* cnt, void* o, cudaStream_t st) {
+  const int G = s->Hq / s->Hkv;
+  const int rows_tok = 128 / G;
+  CUtensorMap mq;
+  int rc;
+  if ((rc = make_map(&mq, q, s->L, s->Hq, s->q_tok_stride, s->q_head_stride, G, rows_tok))) return rc;
+  FlashParams p{};
+  p.L = s->L;
+  p.Hq = s->Hq;
+  p.Hkv = s->Hkv;
+  p.G = G;
+  p.nb = s->L / 64;
+  p.list_len = s->topk + s->recent;
+  p.mtiles = (64 * G) / 128;
+  p.rows_tok = rows_tok;
+  p.scale_log2 = scale_log2(s->d);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.kv_tok = s->kv_tok_stride;
+  p.kv_head = s->kv_head_stride;
+  p.idx = idx;
+  p.cnt = cnt;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_tok = s->q_tok_stride;
+  p.o_head = s->q_head_stride;
+  p.limit_ns = g_wait_limit_ns;
+  p.flags = g_flags;
+  static int attr = set_smem(flash_fwd_kernel<FLASH_SPARSE>, FL_SMEM_SPARSE);
+  if (attr) return attr;
+  const unsigned grid = static_cast<unsigned>(p.nb * s->Hkv * p.mtiles);
+  flash_fwd_kernel<FLASH_SPARSE><<<grid, 256, FL_SMEM_SPARSE, st>>>(mq, mq, mq, p);
+  return launched();
+}
+
+int n_cand(const hs2_shape* s, int b) { return std::max(0, std::min(s->L, 64 * (b + 1)) - s->recent); }
+
+template <int G>
+int launch_importance_g(const CUtensorMap& mq, const CUtensorMap& mk, const ImpParams& p, dim3 grid,
+                        cudaStream_t st) {
+  static int attr = set_smem(importance_kernel<G>, imp_smem_bytes(G));
+  if (attr) return attr;
+  importance_kernel<G><<<grid, 256, imp_smem_bytes(G), st>>>(mq, mk, p);
+  return launched();
+}
+
+int launch_importance(const hs2_shape* s, const void* q, const void* k, const float* lse, int b0, int b1,
+                      float* imp, int64_t row_stride, int skip_le, cudaStream_t st) {
+  const int G = s->Hq / s->Hkv;
+  const int longest = n_cand(s, b1 - 1);
+  if (longest <= 0 || longest <= skip_le) return HS2_OK;
+  CUtensorMap mq, mk;
+  int rc;
+  if ((rc = make_map(&mq, q, s->L, s->Hq, s->q_tok_stride, s->q_head_stride, G, 64))) return rc;
+  if ((rc = make_map(&mk, k, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+  ImpParams p{};
+  p.L = s->L;
+  p.Hq = s->Hq;
+  p.Hkv = s->Hkv;
+  p.G = G;
+  p.recent = s->recent;
+  p.b0 = b0;
+  p.nbs = b1 - b0;
+  p.skip_le = skip_le;
+  p.scale_log2 = scale_log2(s->d);
+  p.lse = lse;
+  p.imp = imp;
+  p.row_stride = row_stride;
+  p.limit_ns = g_wait_limit_ns;
+  p.flags = g_flags;
+  const dim3 grid(static_cast<unsigned>((longest + IMP_CK - 1) / IMP_CK), static_cast<unsigned>(s->Hkv * (b1 - b0)));
+  switch (G) {
+    case 2: return launch_importance_g<2>(mq, mk, p, grid, st);
+    case 4: return launch_importance_g<4>(mq, mk, p, grid, st);
+    case 8: return launch_importance_g<8>(mq, mk, p, grid, st);
+    default: return HS2_ERR_UNSUPPORTED;
+  }
+}
+
+int launch_select(const hs2_shape* s, const float* imp, int64_t row_stride, int b0, int b1, int32_t* idx,
+                  int32_t* cnt, cudaStream_t st) {
+  SelParams p{};
+  p.L = s->L;
+  p.Hkv = s->Hkv;
+  p.nb = s->L / 64;
+  p.recent = s->recent;
+  p.topk = s->topk;
+  p.b0 = b0;
+  p.nbs = b1 - b0;
+  p.list_len = s->topk + s->recent;
+  p.imp = imp;
+  p.row_stride = row_stride;
+  p.idx = idx;
+  p.cnt = cnt;
+  topk_select_kernel<<<static_cast<unsigned>(s->Hkv * (b1 - b0)), SEL_THREADS, 0, st>>>(p);
+  return launched();
+}
+
+int64_t strip_stride(const hs2_shape* s, int b_last) {
+  const int64_t n = n_cand(s, b_last);
+  return std::max<int64_t>(64, (n + 63) / 64 * 64);
+}
+
+size_t min_workspace(const hs2_shape* s) {
+  return static_cast<size_t>(s->Hkv) * static_cast<size_t>(strip_stride(s, s->L / 64 - 1)) * 4u;
+}
+
+constexpr size_t kStripCap = size_t(64) << 20;  // keep one strip L2-resident
+
+size_t recommended_workspace(const hs2_shape* s) {
+  size_t whole = 0;
+  const int nb = s->L / 64;
+  for (int b = 0; b < nb; ++b) whole += static_cast<size_t>(s->Hkv) * strip_stride(s, b) * 4u;
+  return std::max(min_workspace(s), std::min(whole, kStripCap));
+}
+
+}  // namespace
+}  // namespace hs2
+
+using namespace hs2;
+
+extern "C" {
+
+const char* hs2_strerror(int code) {
+  switch (code) {
+    case HS2_OK: return "ok";
+    case HS2_ERR_INVALID_ARG: return "invalid argument";
+    case HS2_ERR_UNSUPPORTED: return "unsupported shape, dtype or alignment";
+    case HS2_ERR_WORKSPACE: return "workspace too small";
+    case HS2_ERR_CUDA: return "CUDA error";
+    case HS2_ERR_TIMEOUT: return "device wait timed out";
+    case HS2_ERR_INDEX: return "index list entry out of range";
+    default: return "unknown hs2 status";
+  }
+}
+
+int hs2_version(void) { return 100; }
+
+uint64_t hs2_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int hs2_debug_set(uint64_t wait_limit_ns, uint32_t flags) {
+  if (wait_limit_ns == 0) return HS2_ERR_INVALID_ARG;
+  g_wait_limit_ns = wait_limit_ns;
+  g_flags = flags;
+  return HS2_OK;
+}
+
+int hs2_attn_fwd(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
+                 const float* v_scale, void* o, float* lse, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if ((rc = check_kv(shape, k, v, k_scale, v_scale))) return rc;
+  if (!q || !o || !lse) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse)) return HS2_ERR_UNSUPPORTED;
+  return launch_attn_fwd(shape, q, k, v, o, lse, static_cast<cudaStream_t>(stream));
+}
+
+int hs2_importance(const hs2_shape* shape, const void* q, const void* k, const float* k_scale, const float* lse,
+                   int32_t b0, int32_t b1, float* imp, int64_t row_stride, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if ((rc = check_kv(shape, k, k, k_scale, k_scale))) return rc;
+  if (!q || !lse || !imp) return HS2_ERR_INVALID_ARG;
+  const int nb = shape->L / 64;
+  if (b0 < 0 || b1 > nb || b0 >= b1) return HS2_ERR_INVALID_ARG;
+  if (row_stride % 4 || row_stride < n_cand(shape, b1 - 1)) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(imp)) return HS2_ERR_UNSUPPORTED;
+  return launch_importance(shape, q, k, lse, b0, b1, imp, row_stride, -1, static_cast<cudaStream_t>(stream));
+}
+
+int hs2_topk_select(const hs2_shape* shape, const float* imp, int64_t row_stride, int32_t b0, int32_t b1,
+                    int32_t* idx, int32_t* cnt, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!imp || !idx || !cnt) return HS2_ERR_INVALID_ARG;
+  const int nb = shape->L / 64;
+  if (b0 < 0 || b1 > nb || b0 >= b1) return HS2_ERR_INVALID_ARG;
+  if (row_stride % 4 || row_stride < n_cand(shape, b1 - 1)) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(imp)) return HS2_ERR_UNSUPPORTED;
+  return launch_select(shape, imp, row_stride, b0, b1, idx, cnt, static_cast<cudaStream_t>(stream));
+}
+
+int hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
+                         const float* v_scale, void* o, float* lse, int32_t* idx, int32_t* cnt, void* workspace,
+                         size_t* workspace_bytes, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!workspace_bytes) return HS2_ERR_INVALID_ARG;
+  if (!workspace) {
+    *workspace_bytes = recommended_workspace(shape);
+    return HS2_OK;
+  }
+  if ((rc = check_kv(shape, k, v, k_scale, v_scale))) return rc;
+  if (!q || !o || !lse || !idx || !cnt) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || !aligned16(workspace)) return HS2_ERR_UNSUPPORTED;
+  const size_t ws = *workspace_bytes;
+  if (ws < min_workspace(shape)) return HS2_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = launch_attn_fwd(shape, q, k, v, o, lse, st))) return rc;
+
+  // Strips of query blocks.  Blocks whose candidates all fit in the top-k
+  // need no importance; the rest are grouped so that a strip's rows
+  // (Hkv x blocks x stride floats) fit the workspace.
+  float* imp = static_cast<float*>(workspace);
+  const int nb = shape->L / 64;
+  int b = 0;
+  while (b < nb) {
+    int b1 = b + 1;
+    if (n_cand(shape, b) <= shape->topk) {
+      while (b1 < nb && n_cand(shape, b1) <= shape->topk) ++b1;
+      if ((rc = launch_select(shape, imp, 64, b, b1, idx, cnt, st))) return rc;
+    } else {
+      while (b1 < nb && static_cast<size_t>(shape->Hkv) * (b1 + 1 - b) * strip_stride(shape, b1) * 4u <= ws) ++b1;
+      const int64_t stride = strip_stride(shape, b1 - 1);
+      if ((rc = launch_importance(shape, q, k, lse, b, b1, imp, stride, shape->topk, st))) return rc;
+      if ((rc = launch_select(shape, imp, stride, b, b1, idx, cnt, st))) return rc;
+    }
+    b = b1;
+  }
+  return HS2_OK;
+}
+
+int hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
+                    const float* v_scale, const int32_t* idx, const int32_t* cnt, void* o, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if ((rc = check_kv(shape, k, v, k_scale, v_scale))) return rc;
+  if (!q || !o || !idx || !cnt) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(idx)) return HS2_ERR_UNSUPPORTED;
+  return launch_sparse(shape, q, k, v, idx, cnt, o, static_cast<cudaStream_t>(stream));
+}
+
+int hs2_sync(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = cudaStreamSynchronize(st);
+  DevStatus ds{};
+  DevStatus zero{};
+  if (cudaMemcpyFromSymbol(&ds, g_status, sizeof(ds)) != cudaSuccess) return HS2_ERR_CUDA;
+  if (ds.code != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return HS2_ERR_CUDA;
+  if (ds.code != 0) return ds.code;
+  return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+}
+
+}  // extern "C"

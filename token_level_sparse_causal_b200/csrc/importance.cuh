@@ -1,0 +1,226 @@
+// Kernel (2): block importance from the full layer's scores.
+//
+// For query block b (64 tokens), KV head g and every candidate key
+// j in C_b = [0, e_b - recent):
+//     I_j = sum_{h in group g} sum_{i in block b} exp(s_hij - lse_hi)
+// (HySparse2 architecture summary, ablation paragraph: the full layer's
+// complete attention scores choose the tokens; the aggregation is this
+// library's reading.)  Because every candidate lies before the block's
+// recent window and recent >= 64, j < i holds for all of the block's
+// queries and no causal mask is needed.
+//
+// Mapping: keys sit on the MMA M dimension.  D = K_tile (128 keys x d) *
+// Q_block^T (d x 64G query-head rows), so TMEM lane r holds key r's scores
+// against every (query, head) of the block, and the thread that owns lane r
+// sums exp2(s * log2e/sqrt(d) - lse_n * log2e) along its row.  The 64G
+// columns are split in sub-tiles of N = min(256, 64G); two TMEM buffers let
+// the tensor core fill one sub-tile while the epilogue drains the other.
+//
+// CTA = 8 warps: warp 0 TMA (Q block once, then K tiles), warp 1 MMA issue
+// and TMEM owner, warps 4-7 epilogue (thread r <-> key r of the tile).
+// Work item = (KV head, block, chunk of IMP_CK keys); the grid is
+// (chunks of the longest row of the strip) x (Hkv * blocks).
+#pragma once
+
+#include "common.cuh"
+#include "flash.cuh"
+
+namespace hs2 {
+
+constexpr int IMP_CK = 2048;   // keys per CTA
+constexpr int IMP_STAGES = 2;  // K tile ring
+
+struct ImpParams {
+  int L, Hq, Hkv, G, recent, b0, nbs;
+  int skip_le;       // rows with |C_b| <= skip_le are not computed (-1: compute all)
+  float scale_log2;  // log2(e) / sqrt(d)
+  const float* lse;  // [Hq][L]
+  float* imp;
+  int64_t row_stride;
+  uint64_t limit_ns;
+  uint32_t flags;
+};
+
+struct ImpBars {
+  uint64_t q_full;
+  uint64_t k_full[IMP_STAGES];
+  uint64_t k_empty[IMP_STAGES];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t fin;
+  uint32_t tmem_slot;
+  int abort;
+};
+
+__host__ __device__ constexpr uint32_t imp_q_bytes(int G) { return static_cast<uint32_t>(64 * G) * 256u; }
+__host__ __device__ constexpr uint32_t imp_kv_off(int G) { return imp_q_bytes(G); }
+__host__ __device__ constexpr uint32_t imp_bar_off(int G) { return imp_q_bytes(G) + IMP_STAGES * TILE_BYTES; }
+__host__ __device__ constexpr uint32_t imp_lse_off(int G) { return imp_bar_off(G) + 256; }
+__host__ __device__ constexpr uint32_t imp_smem_bytes(int G) {
+  return imp_lse_off(G) + static_cast<uint32_t>(64 * G) * 4u + 1024u;
+}
+
+template <int G>
+__global__ void __launch_bounds__(256, 1)
+    importance_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const ImpParams p) {
+  constexpr int NQ = 64 * G;                    // query-head rows of a block
+  constexpr int NSUB = (NQ < 256) ? NQ : 256;   // MMA N per sub-tile
+  constexpr int SUBS = NQ / NSUB;
+  constexpr uint32_t QHALF = static_cast<uint32_t>(NQ) * 128u;
+  constexpr uint32_t IDESC = idesc_bf16_f32(128, NSUB, 0, 0);
+  constexpr uint32_t TMEM_COLS = (2 * NSUB <= 256) ? 256u : 512u;
+
+  const int y = blockIdx.y;
+  const int g = y / p.nbs;
+  const int b = p.b0 + y % p.nbs;
+  const int e_b = min(p.L, 64 * (b + 1));
+  const int n_c = max(0, e_b - p.recent);
+  const int j0 = static_cast<int>(blockIdx.x) * IMP_CK;
+  if (j0 >= n_c || n_c <= p.skip_le) return;  // uniform exit before any allocation
+  const int ntiles = (min(IMP_CK, n_c - j0) + 127) / 128;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  ImpBars* bars = reinterpret_cast<ImpBars*>(smem + imp_bar_off(G));
+  float* nlse = reinterpret_cast<float*>(smem + imp_lse_off(G));
+  const uint32_t q_base = smem_u32(smem);
+  const uint32_t k_base = smem_u32(smem + imp_kv_off(G));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &bars->abort;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < IMP_STAGES; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->acc_full[s], 1);
+      mbar_init(&bars->acc_empty[s], 128);
+    }
+    mbar_init(&bars->fin, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  // -lse * log2(e) for every (query, head) column n = t * G + hl of the block
+  for (int n = threadIdx.x; n < NQ; n += blockDim.x) {
+    const int t = n / G, hl = n % G;
+    nlse[n] = -p.lse[static_cast<int64_t>(g * G + hl) * p.L + 64 * b + t] * 1.44269504088896340736f;
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0 && !(p.flags & FLAG_SKIP_LOADS)) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      mbar_arrive_expect_tx(&bars->q_full, 2 * QHALF);
+      tma_load_3d(smem, &tmQ, &bars->q_full, 0, g * G, 64 * b);
+      tma_load_3d(smem + QHALF, &tmQ, &bars->q_full, 64, g * G, 64 * b);
+      int last = -1;
+      for (int t = 0; t < ntiles; ++t) {
+        const int s = t % IMP_STAGES;
+        if (t >= IMP_STAGES &&
+            !mbar_wait(&bars->k_empty[s], ((t / IMP_STAGES) - 1) & 1, p.limit_ns, abort_flag, 201))
+          break;
+        uint8_t* kd = smem + imp_kv_off(G) + s * TILE_BYTES;
+        mbar_arrive_expect_tx(&bars->k_full[s], TILE_BYTES);
+        tma_load_3d(kd, &tmK, &bars->k_full[s], 0, g, j0 + t * 128);
+        tma_load_3d(kd + HALF_BYTES, &tmK, &bars->k_full[s], 64, g, j0 + t * 128);
+        last = t;
+      }
+      for (int t = max(0, last - IMP_STAGES + 1); t <= last; ++t)
+        wait_done(&bars->k_full[t % IMP_STAGES], (t / IMP_STAGES) & 1, p.limit_ns, 202);
+      wait_done(&bars->q_full, 0, p.limit_ns, 203);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = mbar_wait(&bars->q_full, 0, p.limit_ns, abort_flag, 211);
+      if (ok) tc_fence_after();
+      int u = 0;
+      for (int t = 0; t < ntiles && ok; ++t) {
+        const int s = t % IMP_STAGES;
+        if (!mbar_wait(&bars->k_full[s], (t / IMP_STAGES) & 1, p.limit_ns, abort_flag, 212)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t kb = k_base + s * TILE_BYTES;
+        for (int sub = 0; sub < SUBS; ++sub, ++u) {
+          const int buf = u & 1;
+          if (u >= 2 && !mbar_wait(&bars->acc_empty[buf], ((u >> 1) - 1) & 1, p.limit_ns, abort_flag, 213)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + buf * NSUB;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+            const uint32_t qoff = (kk >> 2) * QHALF + sub * NSUB * 128 + (kk & 3) * 32;
+            umma_ss(d, sdesc_sw128(kb + koff, 16, 1024), sdesc_sw128(q_base + qoff, 16, 1024), IDESC,
+                    kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars->acc_full[buf]);
+        }
+        if (ok) umma_commit(&bars->k_empty[s]);
+      }
+      umma_commit(&bars->fin);
+      wait_done(&bars->fin, 0, p.limit_ns, 214);
+    }
+  } else if (warp >= 4) {
+    const int r = threadIdx.x - 128;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    float* out = p.imp + (static_cast<int64_t>(g) * p.nbs + (b - p.b0)) * p.row_stride;
+    const float c2 = p.scale_log2;
+    int u = 0;
+    bool ok = true;
+    for (int t = 0; t < ntiles && ok; ++t) {
+      float acc = 0.f;
+      for (int sub = 0; sub < SUBS; ++sub, ++u) {
+        const int buf = u & 1;
+        if (!warp_wait(&bars->acc_full[buf], (u >> 1) & 1, p.limit_ns, abort_flag, 221)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float4* nl4 = reinterpret_cast<const float4*>(nlse + sub * NSUB);
+#pragma unroll 1
+        for (int c = 0; c < NSUB / 32; ++c) {
+          uint32_t sr[32];
+          tmem_ld32(tmem + lane_off + buf * NSUB + c * 32, sr);
+          tmem_ld_wait();
+          reg_fence(sr);
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 nl = nl4[c * 8 + e4];  // broadcast read
+            acc += ex2_approx(fmaf(__uint_as_float(sr[4 * e4 + 0]), c2, nl.x));
+            acc += ex2_approx(fmaf(__uint_as_float(sr[4 * e4 + 1]), c2, nl.y));
+            acc += ex2_approx(fmaf(__uint_as_float(sr[4 * e4 + 2]), c2, nl.z));
+            acc += ex2_approx(fmaf(__uint_as_float(sr[4 * e4 + 3]), c2, nl.w));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->acc_empty[buf]);
+      }
+      const int j = j0 + t * 128 + r;
+      if (ok && j < n_c) out[j] = acc;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace hs2

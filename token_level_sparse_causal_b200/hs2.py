@@ -1,0 +1,162 @@
+"""Thin ctypes binding over libhs2.so (argument marshalling only).
+
+Every step of the prefill path runs in the library's CUDA kernels; this
+module only turns torch tensors into device pointers and sizes, picks the
+current CUDA stream, and raises Hs2Error on a non-zero status.  If the shared
+library is missing or fails to load, importing the functions raises: there is
+no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhs2.so")
+
+HS2_OK, HS2_ERR_INVALID_ARG, HS2_ERR_UNSUPPORTED, HS2_ERR_WORKSPACE, HS2_ERR_CUDA, HS2_ERR_TIMEOUT, HS2_ERR_INDEX = range(7)
+HS2_KV_BF16, HS2_KV_E4M3 = 0, 1
+
+EXPORTS = ("hs2_full_attn_select", "hs2_sparse_attn", "hs2_sync", "hs2_attn_fwd", "hs2_importance",
+           "hs2_topk_select", "hs2_strerror", "hs2_debug_set", "hs2_version", "hs2_launch_count")
+
+
+class Hs2Shape(ctypes.Structure):
+    _fields_ = [("L", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("block", ctypes.c_int32), ("topk", ctypes.c_int32), ("recent", ctypes.c_int32),
+                ("kv_dtype", ctypes.c_int32), ("q_tok_stride", ctypes.c_int64), ("q_head_stride", ctypes.c_int64),
+                ("kv_tok_stride", ctypes.c_int64), ("kv_head_stride", ctypes.c_int64)]
+
+
+class Hs2Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: hs2 status {code} ({strerror(code)})")
+        self.code = code
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+_vp, _i32, _i64, _u32, _u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64
+_SIGS = {
+    "hs2_full_attn_select": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                             ctypes.POINTER(ctypes.c_size_t), _vp],
+    "hs2_sparse_attn": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "hs2_sync": [_vp],
+    "hs2_attn_fwd": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "hs2_importance": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i64, _vp],
+    "hs2_topk_select": [ctypes.POINTER(Hs2Shape), _vp, _i64, _i32, _i32, _vp, _vp, _vp],
+    "hs2_debug_set": [_u64, _u32],
+    "hs2_version": [],
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libhs2.so (built in-tree by token_level_sparse_causal_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libhs2.so not built at {LIB_PATH}; run token_level_sparse_causal_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, args in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.hs2_launch_count.argtypes = []
+        L.hs2_launch_count.restype = ctypes.c_uint64
+        L.hs2_strerror.argtypes = [ctypes.c_int]
+        L.hs2_strerror.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().hs2_strerror(int(code)).decode()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != HS2_OK:
+        raise Hs2Error(rc, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def make_shape(q: torch.Tensor, k: torch.Tensor, topk: int = 1024, recent: int = 128, block: int = 64,
+               kv_dtype: int = HS2_KV_BF16) -> Hs2Shape:
+    """hs2_shape for Q [L][Hq][d] and K [L][Hkv][d] tensors (element strides)."""
+    L, Hq, d = q.shape
+    return Hs2Shape(L=L, Hq=Hq, Hkv=k.shape[1], d=d, block=block, topk=topk, recent=recent, kv_dtype=kv_dtype,
+                    q_tok_stride=q.stride(0), q_head_stride=q.stride(1), kv_tok_stride=k.stride(0),
+                    kv_head_stride=k.stride(1))
+
+
+def workspace_bytes(shape: Hs2Shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().hs2_full_attn_select(ctypes.byref(shape), None, None, None, None, None, None, None, None, None,
+                                      None, ctypes.byref(n), None), "hs2_full_attn_select(size query)")
+    return int(n.value)
+
+
+def hs2_full_attn_select(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, workspace, stream=None) -> None:
+    n = ctypes.c_size_t(workspace.numel() * workspace.element_size())
+    _check(lib().hs2_full_attn_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale),
+                                      _ptr(o), _ptr(lse), _ptr(idx), _ptr(cnt), _ptr(workspace), ctypes.byref(n),
+                                      _stream(stream)), "hs2_full_attn_select")
+
+
+def hs2_sparse_attn(shape, q, k, v, k_scale, v_scale, idx, cnt, o, stream=None) -> None:
+    _check(lib().hs2_sparse_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale),
+                                 _ptr(idx), _ptr(cnt), _ptr(o), _stream(stream)), "hs2_sparse_attn")
+
+
+def hs2_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, stream=None) -> None:
+    _check(lib().hs2_attn_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale),
+                              _ptr(o), _ptr(lse), _stream(stream)), "hs2_attn_fwd")
+
+
+def hs2_importance(shape, q, k, k_scale, lse, b0, b1, imp, row_stride, stream=None) -> None:
+    _check(lib().hs2_importance(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(k_scale), _ptr(lse), int(b0), int(b1),
+                                _ptr(imp), int(row_stride), _stream(stream)), "hs2_importance")
+
+
+def hs2_topk_select(shape, imp, row_stride, b0, b1, idx, cnt, stream=None) -> None:
+    _check(lib().hs2_topk_select(ctypes.byref(shape), _ptr(imp), int(row_stride), int(b0), int(b1), _ptr(idx),
+                                 _ptr(cnt), _stream(stream)), "hs2_topk_select")
+
+
+def hs2_sync(stream=None) -> None:
+    _check(lib().hs2_sync(_stream(stream)), "hs2_sync")
+
+
+def hs2_launch_count() -> int:
+    return int(lib().hs2_launch_count())
+
+
+def hs2_debug_set(wait_limit_ns: int = 2_000_000_000, flags: int = 0) -> None:
+    _check(lib().hs2_debug_set(int(wait_limit_ns), int(flags)), "hs2_debug_set")
+
+
+# ------------------------------------------------------------ conveniences --
+
+def alloc_outputs(shape: Hs2Shape, q: torch.Tensor, with_workspace: bool = True) -> dict:
+    """Device buffers for one full-layer call (torch supplies the memory)."""
+    dev = q.device
+    nb = shape.L // shape.block
+    out = {
+        "o": torch.empty_like(q),
+        "lse": torch.empty((shape.Hq, shape.L), device=dev, dtype=torch.float32),
+        "idx": torch.empty((shape.Hkv, nb, shape.topk + shape.recent), device=dev, dtype=torch.int32),
+        "cnt": torch.empty((shape.Hkv, nb), device=dev, dtype=torch.int32),
+    }
+    if with_workspace:
+        out["workspace"] = torch.empty(workspace_bytes(shape) // 4 + 4, device=dev, dtype=torch.float32)
+    return out
