@@ -16,6 +16,7 @@
 #include <stdint.h>
 
 #include "../../include/hs2.h"
+#include "exp2_poly.cuh"
 
 namespace hs2 {
 
@@ -53,6 +54,30 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipes (for x >= -125; smaller x gives about 2^-125):
+// 2^x = 2^j * 2^f with j = round(x) and f = x - j in [-1/2, 1/2] (Cody-Waite
+// style reduction), 2^f from a degree-3 relative-minimax polynomial derived
+// by derive_exp2_poly.py (max relative error 7.5e-5), and 2^j added straight
+// into the exponent field.  Adding 1.5 * 2^23 rounds x to an integer held in
+// the low mantissa bits of t, and (bits(t) << 23) is j << 23 modulo 2^32.
+__device__ __forceinline__ float exp2_fma3(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(EXP2_D3_C3, f, EXP2_D3_C2), f, EXP2_D3_C1), f, EXP2_D3_C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Same with the degree-4 polynomial (max relative error 2.6e-6).
+__device__ __forceinline__ float exp2_fma4(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p =
+      fmaf(fmaf(fmaf(fmaf(EXP2_D4_C4, f, EXP2_D4_C3), f, EXP2_D4_C2), f, EXP2_D4_C1), f, EXP2_D4_C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
