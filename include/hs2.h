@@ -99,6 +99,34 @@ int hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, c
                          int32_t* cnt, void* workspace, size_t* workspace_bytes, void* stream);
 
 /*
+ * hs2_full_attn_select without a caller workspace.  (The paper has no
+ * counterpart: this is a deployment convenience.)
+ *
+ * For callers that cannot allocate device memory where they call this: a
+ * plugin inside a host framework that owns the whole device pool and hands
+ * plugins only the pointers of their tensors, or a latency-critical path where
+ * a cudaMalloc could synchronise the device.  The importance strips live in a
+ * fixed 16 MiB array inside the library (a file-scope __device__ array, held on
+ * every GPU that loads the library until the process exits); nothing is
+ * allocated or freed.
+ *
+ *   - Shapes whose one-block strip needs more than 16 MiB
+ *     (Hkv * roundup(L - recent, 64) * 4 bytes > 16 MiB, e.g. L = 1M with
+ *     Hkv = 8) return HS2_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current; make that first call before any stream capture, and pass
+ *     a stream of the current device.
+ *   - Every call shares the one array, which keeps the previous call's
+ *     contents; nothing in it has to start at zero (each importance entry the
+ *     select reads is written earlier in the same call).  Calls that overlap on
+ *     the GPU (e.g. on two streams of one device) race on it: serialise them.
+ * Results equal those of hs2_full_attn_select on the same inputs.
+ */
+int hs2_full_attn_select_static(const hs2_shape* shape, const void* q, const void* k, const void* v,
+                                const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,
+                                int32_t* cnt, void* stream);
+
+/*
  * One sparse layer (KV Reuse): for every query i of block b and head h,
  * softmax over the listed positions j <= i of q_hi . k_j / sqrt(d), times V,
  * using the shared K/V and the index lists written by hs2_full_attn_select.

@@ -260,6 +260,30 @@ size_t recommended_workspace(const hs2_shape* s) {
   return std::max(min_workspace(s), std::min(whole, kStripCap));
 }
 
+// Scratch for hs2_full_attn_select_static: the importance strips of callers
+// that cannot allocate.  Host code must not use the symbol as an address; the
+// device address is looked up per device with cudaGetSymbolAddress.
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+__device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[128] = {};
+
+// Device address of g_static_scratch on the current device (looked up once per
+// device, with that device current).
+int static_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return HS2_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return HS2_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return HS2_OK;
+}
+
 }  // namespace
 }  // namespace hs2
 
@@ -364,6 +388,18 @@ int hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, c
     b = b1;
   }
   return HS2_OK;
+}
+
+int hs2_full_attn_select_static(const hs2_shape* shape, const void* q, const void* k, const void* v,
+                                const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,
+                                int32_t* cnt, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (min_workspace(shape) > kStaticScratchBytes) return HS2_ERR_WORKSPACE;  // before any CUDA call
+  void* scratch = nullptr;
+  if ((rc = static_scratch(&scratch))) return rc;
+  size_t n = kStaticScratchBytes;
+  return hs2_full_attn_select(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, scratch, &n, stream);
 }
 
 int hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,

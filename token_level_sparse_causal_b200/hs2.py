@@ -20,7 +20,8 @@ HS2_OK, HS2_ERR_INVALID_ARG, HS2_ERR_UNSUPPORTED, HS2_ERR_WORKSPACE, HS2_ERR_CUD
 HS2_KV_BF16, HS2_KV_E4M3 = 0, 1
 
 EXPORTS = ("hs2_full_attn_select", "hs2_sparse_attn", "hs2_sync", "hs2_attn_fwd", "hs2_importance",
-           "hs2_topk_select", "hs2_strerror", "hs2_debug_set", "hs2_version", "hs2_launch_count")
+           "hs2_topk_select", "hs2_strerror", "hs2_debug_set", "hs2_version", "hs2_launch_count",
+           "hs2_full_attn_select_static")
 
 
 class Hs2Shape(ctypes.Structure):
@@ -42,6 +43,7 @@ _vp, _i32, _i64, _u32, _u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, c
 _SIGS = {
     "hs2_full_attn_select": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                              ctypes.POINTER(ctypes.c_size_t), _vp],
+    "hs2_full_attn_select_static": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "hs2_sparse_attn": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "hs2_sync": [_vp],
     "hs2_attn_fwd": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
@@ -111,6 +113,14 @@ def hs2_full_attn_select(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, wor
     _check(lib().hs2_full_attn_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale),
                                       _ptr(o), _ptr(lse), _ptr(idx), _ptr(cnt), _ptr(workspace), ctypes.byref(n),
                                       _stream(stream)), "hs2_full_attn_select")
+
+
+def hs2_full_attn_select_static(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, stream=None) -> None:
+    """Same as hs2_full_attn_select, scratch taken from the library's fixed
+    16 MiB device array (for callers that cannot allocate)."""
+    _check(lib().hs2_full_attn_select_static(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale),
+                                             _ptr(v_scale), _ptr(o), _ptr(lse), _ptr(idx), _ptr(cnt),
+                                             _stream(stream)), "hs2_full_attn_select_static")
 
 
 def hs2_sparse_attn(shape, q, k, v, k_scale, v_scale, idx, cnt, o, stream=None) -> None:
