@@ -182,6 +182,14 @@ const char* hs2_strerror(int code);
  */
 int hs2_debug_set(uint64_t wait_limit_ns, uint32_t flags);
 
+/*
+ * Evaluates, on the device, the exponentials the kernels use for x[0..n):
+ * y_mufu = hardware ex2.approx, y_fma3 / y_fma4 = the software 2^x on the FMA
+ * pipes (degree-3 and degree-4 polynomials; valid for x >= -125).  Device
+ * pointers, n >= 0; for checking their error against an fp64 reference.
+ */
+int hs2_exp2_check(const float* x, float* y_mufu, float* y_fma3, float* y_fma4, int64_t n, void* stream);
+
 /* Library version as major * 10000 + minor * 100 + patch. */
 int hs2_version(void);
 

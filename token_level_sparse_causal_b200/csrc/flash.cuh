@@ -2,36 +2,42 @@
 // pipeline:
 //
 //   FLASH_DENSE  -- kernel (1): causal grouped-query attention of the full
-//                   layer, one CTA per (128-query tile, query head), K/V tiles
-//                   of 128 keys streamed by TMA; writes O and the per-query
-//                   natural-log LSE.  (HySparse2 architecture summary, ablation
-//                   paragraph: the full layer's complete scores; SHARP
-//                   walk-through, section 1.1: softmax(Q K^T / sqrt(d)) V.)
+//                   layer, one CTA per (pair of 128-query tiles, query head),
+//                   K/V tiles of 128 keys streamed by TMA; writes O and the
+//                   per-query natural-log LSE.  (HySparse2 architecture
+//                   summary, ablation paragraph: the full layer's complete
+//                   scores; SHARP walk-through, section 1.1:
+//                   softmax(Q K^T / sqrt(d)) V.)
 //   FLASH_SPARSE -- kernel (4): a sparse layer (KV Reuse, KV-sharing
-//                   paragraph), one CTA per (query block b, KV head g, 128-row
-//                   M tile); the 128 rows are (128/G tokens) x (G heads) of the
-//                   block, all sharing the block's index list, whose K/V rows
-//                   are gathered with 16-byte cp.async into swizzled shared
-//                   memory; the causal mask j <= i applies to listed positions.
+//                   paragraph), one CTA per (query block b, KV head g, pair of
+//                   128-row M tiles); each M tile is (128/G tokens) x (G heads)
+//                   of the block, all sharing the block's index list, whose K/V
+//                   rows are gathered with 16-byte cp.async into swizzled
+//                   shared memory; the causal mask j <= i applies to listed
+//                   positions.
 //
-// CTA = 8 warps:
-//   warp 0      TMA: Q tile (both modes), K/V tiles (dense)
+// CTA = 12 warps:
+//   warp 0      TMA: Q tiles (both modes), K/V tiles (dense)
 //   warp 1      TMEM allocation; one thread issues every tcgen05.mma
 //   warps 2-3   K/V gather (sparse)
-//   warps 4-7   softmax, O rescale and epilogue; thread r owns row r (TMEM
-//               lane r) of S, P and O
+//   warps 4-7   softmax / rescale / epilogue of query tile A (thread r <-> row r)
+//   warps 8-11  the same for query tile B
 //
-// Tensor memory (512 columns): S0 = [0,128), S1 = [128,256), O = [256,384).
-// P (bf16) is written over the first 64 columns of the S buffer it came from
-// and fed to the PV product straight from tensor memory.
+// Tensor memory (512 columns): S_A [0,128), S_B [128,256), O_A [256,384),
+// O_B [384,512).  P (bf16) is written over the first 64 columns of its S and
+// fed to the PV product straight from tensor memory.
 //
-// Per key tile j:  S_j = Q K_j^T (SS MMA, M=N=128, K=d=128 in 8 steps);
-// softmax rows in the log2 domain with a lazily updated reference max: O is
-// rescaled only when the running max grows by more than 2^8, so P stays
-// below 256 and the final O / l is exact up to rounding; O += P_j V_j (TS
-// MMA, V as an MN-major operand).  Issue order of the MMA thread is
-// S_0, S_1, PV_0, S_2, PV_1, ... so the tensor core works on S_{j+1} while
-// the softmax warps process S_j.
+// Per key tile j the MMA thread issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1),
+// so while softmax A works on S_A(j+1) the tensor core runs PV_B(j) and
+// S_B(j+1), and vice versa: the two softmax warpgroups take turns and the
+// tensor core always has the other tile's work.
+//
+// Softmax runs in the log2 domain with a lazily updated reference max: O is
+// rescaled only when a row max grows by more than 8 (P stays below 256; the
+// final O / l is exact up to rounding).  A quarter of the exponentials of
+// every unmasked tile are computed on the FMA pipes (exp2_fma3) so the MUFU
+// unit stops being the bottleneck; row max and row sum use independent
+// partial accumulators.
 #pragma once
 
 #include "common.cuh"
@@ -40,6 +46,7 @@ namespace hs2 {
 
 constexpr int HD = 128;
 constexpr int FL_STAGES = 2;
+constexpr int FL_THREADS = 384;
 constexpr uint32_t TILE_BYTES = 128u * 128u * 2u;  // one 128 x 128 bf16 tile
 constexpr uint32_t HALF_BYTES = 128u * 64u * 2u;   // its d-half (128 rows x 128 B)
 constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
@@ -50,8 +57,9 @@ constexpr uint32_t FLAG_SKIP_LOADS = 1u;
 constexpr int MAX_LIST = 4096;
 
 struct FlashParams {
-  int L, Hq, Hkv, G, nqt;  // nqt: 128-row query tiles (dense)
+  int L, Hq, Hkv, G, nqt, npairs;      // dense: 128-row query tiles, tile pairs
   int nb, list_len, mtiles, rows_tok;  // sparse: blocks, list stride, M tiles per (b,g), tokens per M tile
+  int mpairs;                          // sparse: pairs of M tiles per (b,g)
   float scale_log2;                    // log2(e) / sqrt(d)
   const __nv_bfloat16* k;              // gather sources (sparse)
   const __nv_bfloat16* v;
@@ -70,17 +78,17 @@ struct FlashBars {
   uint64_t full_k[FL_STAGES];
   uint64_t full_v[FL_STAGES];
   uint64_t empty[FL_STAGES];
-  uint64_t s_full[2];
-  uint64_t p_ready;
-  uint64_t o_done;
+  uint64_t s_full[2];  // per query tile
+  uint64_t p_ready[2];
+  uint64_t o_done[2];
   uint64_t fin;
   uint32_t tmem_slot;
   int abort;
 };
 
-constexpr uint32_t FL_Q_OFF = 0;
-constexpr uint32_t FL_KV_OFF = TILE_BYTES;
-constexpr uint32_t FL_BAR_OFF = TILE_BYTES + FL_STAGES * 2 * TILE_BYTES;
+constexpr uint32_t FL_Q_OFF = 0;                // Q_A, then Q_B
+constexpr uint32_t FL_KV_OFF = 2 * TILE_BYTES;  // stage s: K at +0, V at +TILE_BYTES
+constexpr uint32_t FL_BAR_OFF = FL_KV_OFF + FL_STAGES * 2 * TILE_BYTES;
 constexpr uint32_t FL_POS_OFF = FL_BAR_OFF + 256;
 constexpr uint32_t FL_SMEM_DENSE = FL_POS_OFF + 1024;  // + alignment slack
 constexpr uint32_t FL_SMEM_SPARSE = FL_POS_OFF + MAX_LIST * 4 + 1024;
@@ -93,10 +101,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64
   return __all_sync(0xffffffffu, ok);
 }
 
+// Waits for work already in flight (TMA or MMA completion), ignoring the
+// abort flag: such work always finishes, and the CTA must not release its
+// shared or tensor memory while it is outstanding.
 __device__ __forceinline__ bool wait_done(uint64_t* bar, uint32_t parity, uint64_t limit_ns, int where) {
-  // Waits for work already in flight (TMA or MMA completion), ignoring the
-  // abort flag: such work always finishes, and the CTA must not release its
-  // shared or tensor memory while it is outstanding.
   const uint32_t a = smem_u32(bar);
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
@@ -109,7 +117,7 @@ __device__ __forceinline__ bool wait_done(uint64_t* bar, uint32_t parity, uint64
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(FL_THREADS, 1)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const FlashParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -121,25 +129,30 @@ __global__ void __launch_bounds__(256, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &bars->abort;
 
-  // ---- work item
-  int qt = 0, h = 0, g = 0, b = 0, mt = 0, ntiles = 0, cnt = 0, e_b = 0;
+  // ---- work item: query tiles A and B (B may be absent), key tiles nA / nB
+  int h = 0, g = 0, b = 0, pair = 0, cnt = 0, e_b = 0, nA = 0, nB = 0;
   if (MODE == FLASH_DENSE) {
-    qt = p.nqt - 1 - static_cast<int>(blockIdx.x) / p.Hq;  // longest rows first
+    pair = p.npairs - 1 - static_cast<int>(blockIdx.x) / p.Hq;  // longest rows first
     h = static_cast<int>(blockIdx.x) % p.Hq;
     g = h / p.G;
-    ntiles = qt + 1;
+    nA = 2 * pair + 1;
+    nB = (2 * pair + 1 < p.nqt) ? 2 * pair + 2 : 0;
   } else {
-    mt = static_cast<int>(blockIdx.x) % p.mtiles;
-    const int bg = static_cast<int>(blockIdx.x) / p.mtiles;
+    pair = static_cast<int>(blockIdx.x) % p.mpairs;
+    const int bg = static_cast<int>(blockIdx.x) / p.mpairs;
     g = bg % p.Hkv;
     b = bg / p.Hkv;
     e_b = min(p.L, 64 * (b + 1));
     cnt = p.cnt[static_cast<int64_t>(g) * p.nb + b];
     cnt = max(0, min(cnt, p.list_len));
-    ntiles = (cnt + 127) / 128;
+    const int nt = (cnt + 127) / 128;
+    nA = nt;
+    nB = (2 * pair + 1 < p.mtiles) ? nt : 0;
     const int32_t* list = p.idx + (static_cast<int64_t>(g) * p.nb + b) * p.list_len;
-    for (int i = threadIdx.x; i < ntiles * 128; i += blockDim.x) pos_s[i] = (i < cnt) ? list[i] : -1;
+    for (int i = threadIdx.x; i < nt * 128; i += blockDim.x) pos_s[i] = (i < cnt) ? list[i] : -1;
   }
+  const int n = max(nA, nB);
+  const bool has_b = (MODE == FLASH_DENSE) ? (nB > 0) : (2 * pair + 1 < p.mtiles);
 
   if (threadIdx.x == 0) {
     const uint32_t kv_arrivals = (MODE == FLASH_DENSE) ? 1u : 64u;
@@ -149,10 +162,11 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(&bars->full_v[s], kv_arrivals);
       mbar_init(&bars->empty[s], 1);
     }
-    mbar_init(&bars->s_full[0], 1);
-    mbar_init(&bars->s_full[1], 1);
-    mbar_init(&bars->p_ready, 128);
-    mbar_init(&bars->o_done, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->p_ready[x], 128);
+      mbar_init(&bars->o_done[x], 1);
+    }
     mbar_init(&bars->fin, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -168,20 +182,24 @@ __global__ void __launch_bounds__(256, 1)
 
   if (warp == 0) {
     // =========================================================== TMA loads
-    if (lane == 0 && !(p.flags & FLAG_SKIP_LOADS) && ntiles > 0) {
+    if (lane == 0 && !(p.flags & FLAG_SKIP_LOADS) && n > 0) {
       tma_prefetch_desc(&tmQ);
-      mbar_arrive_expect_tx(&bars->q_full, TILE_BYTES);
-      if (MODE == FLASH_DENSE) {
-        tma_load_3d(smem + FL_Q_OFF, &tmQ, &bars->q_full, 0, h, qt * 128);
-        tma_load_3d(smem + FL_Q_OFF + HALF_BYTES, &tmQ, &bars->q_full, 64, h, qt * 128);
-      } else {
-        const int t0 = 64 * b + mt * p.rows_tok;
-        tma_load_3d(smem + FL_Q_OFF, &tmQ, &bars->q_full, 0, g * p.G, t0);
-        tma_load_3d(smem + FL_Q_OFF + HALF_BYTES, &tmQ, &bars->q_full, 64, g * p.G, t0);
+      const int nq = has_b ? 2 : 1;
+      mbar_arrive_expect_tx(&bars->q_full, static_cast<uint32_t>(nq) * TILE_BYTES);
+      for (int x = 0; x < nq; ++x) {
+        uint8_t* qd = smem + FL_Q_OFF + x * TILE_BYTES;
+        if (MODE == FLASH_DENSE) {
+          tma_load_3d(qd, &tmQ, &bars->q_full, 0, h, (2 * pair + x) * 128);
+          tma_load_3d(qd + HALF_BYTES, &tmQ, &bars->q_full, 64, h, (2 * pair + x) * 128);
+        } else {
+          const int t0 = 64 * b + (2 * pair + x) * p.rows_tok;
+          tma_load_3d(qd, &tmQ, &bars->q_full, 0, g * p.G, t0);
+          tma_load_3d(qd + HALF_BYTES, &tmQ, &bars->q_full, 64, g * p.G, t0);
+        }
       }
       if (MODE == FLASH_DENSE) {
         int last = -1;
-        for (int j = 0; j < ntiles; ++j) {
+        for (int j = 0; j < n; ++j) {
           const int s = j % FL_STAGES;
           if (j >= FL_STAGES &&
               !mbar_wait(&bars->empty[s], ((j / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 101))
@@ -206,47 +224,70 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp == 1) {
     // ========================================================== MMA issue
-    if (lane == 0 && ntiles > 0) {
-      bool ok = mbar_wait(&bars->q_full, 0, p.limit_ns, abort_flag, 111);
-      auto do_pv = [&](int t) -> bool {
-        const int s = t % FL_STAGES;
-        if (!mbar_wait(&bars->p_ready, t & 1, p.limit_ns, abort_flag, 112)) return false;
-        if (!mbar_wait(&bars->full_v[s], (t / FL_STAGES) & 1, p.limit_ns, abort_flag, 113)) return false;
-        tc_fence_after();
-        const uint32_t vb = kv_base + s * 2 * TILE_BYTES + TILE_BYTES;
+    if (lane == 0 && n > 0) {
+      const int nx[2] = {nA, nB};
+      auto issue_s = [&](int x, int j) {
+        const uint32_t kb = kv_base + (j % FL_STAGES) * 2 * TILE_BYTES;
+        const uint32_t qb = q_base + x * TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + x * 128, sdesc_sw128(qb + koff, 16, 1024), sdesc_sw128(kb + koff, 16, 1024), IDESC_S,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars->s_full[x]);
+      };
+      auto issue_pv = [&](int x, int j) {
+        const uint32_t vb = kv_base + (j % FL_STAGES) * 2 * TILE_BYTES + TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bdesc = sdesc_sw128(vb + kk * 2048, HALF_BYTES, 1024);
-          umma_ts(tmem + 256, tmem + (t & 1) * 128 + kk * 8, bdesc, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bdesc, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars->o_done);
-        umma_commit(&bars->empty[s]);
-        return true;
+        umma_commit(&bars->o_done[x]);
       };
+      bool ok = mbar_wait(&bars->q_full, 0, p.limit_ns, abort_flag, 111);
+      if (ok) ok = mbar_wait(&bars->full_k[0], 0, p.limit_ns, abort_flag, 112);
       if (ok) {
         tc_fence_after();
-        for (int j = 0; j < ntiles && ok; ++j) {
-          const int s = j % FL_STAGES;
-          if (!mbar_wait(&bars->full_k[s], (j / FL_STAGES) & 1, p.limit_ns, abort_flag, 114)) {
+        for (int x = 0; x < 2; ++x)
+          if (nx[x] > 0) issue_s(x, 0);
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        const int s = j % FL_STAGES;
+        bool v_ready = false, k_next = false;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (j >= nx[x]) continue;
+          if (!mbar_wait(&bars->p_ready[x], j & 1, p.limit_ns, abort_flag, 113)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t kb = kv_base + s * 2 * TILE_BYTES;
-          const uint32_t d = tmem + (j & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t koff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            umma_ss(d, sdesc_sw128(q_base + koff, 16, 1024), sdesc_sw128(kb + koff, 16, 1024), IDESC_S,
-                    kk > 0 ? 1u : 0u);
+          if (!v_ready) {
+            if (!mbar_wait(&bars->full_v[s], (j / FL_STAGES) & 1, p.limit_ns, abort_flag, 114)) {
+              ok = false;
+              break;
+            }
+            v_ready = true;
           }
-          umma_commit(&bars->s_full[j & 1]);
-          if (j > 0) ok = do_pv(j - 1);
+          tc_fence_after();
+          issue_pv(x, j);
+          if (j + 1 < nx[x]) {
+            if (!k_next) {
+              const int s1 = (j + 1) % FL_STAGES;
+              if (!mbar_wait(&bars->full_k[s1], ((j + 1) / FL_STAGES) & 1, p.limit_ns, abort_flag, 115)) {
+                ok = false;
+                break;
+              }
+              k_next = true;
+              tc_fence_after();
+            }
+            issue_s(x, j + 1);
+          }
         }
-        if (ok) do_pv(ntiles - 1);
+        if (ok) umma_commit(&bars->empty[s]);
       }
       umma_commit(&bars->fin);
-      wait_done(&bars->fin, 0, p.limit_ns, 115);
+      wait_done(&bars->fin, 0, p.limit_ns, 116);
     }
   } else if (warp < 4) {
     // ========================================================= K/V gather
@@ -255,15 +296,17 @@ __global__ void __launch_bounds__(256, 1)
       const int row_sub = (pt >> 4) & 1, chunk = pt & 15, pw = pt >> 5;
       const __nv_bfloat16* kg = p.k + static_cast<int64_t>(g) * p.kv_head + chunk * 8;
       const __nv_bfloat16* vg = p.v + static_cast<int64_t>(g) * p.kv_head + chunk * 8;
-      for (int j = 0; j < ntiles; ++j) {
+      // Per key tile: K rows then V rows as two cp.async groups; K is
+      // published as soon as it lands so S can start while V is in flight.
+      // A tile is published before the next stage is awaited: the MMA order
+      // needs tile j+1's K before it can release tile j's stage.
+      for (int j = 0; j < n; ++j) {
         const int s = j % FL_STAGES;
         if (j >= FL_STAGES &&
             !mbar_wait(&bars->empty[s], ((j / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 121))
           break;
         const uint32_t kd = kv_base + s * 2 * TILE_BYTES;
-        int64_t src[32];
-        uint32_t nbytes[32];
-#pragma unroll
+#pragma unroll 4
         for (int it = 0; it < 32; ++it) {
           const int r = pw * 2 + row_sub + 4 * it;
           const int gi = j * 128 + r;
@@ -271,15 +314,18 @@ __global__ void __launch_bounds__(256, 1)
           const bool listed = gi < cnt;
           const bool valid = listed && pj >= 0 && pj < e_b;
           if (listed && !valid) report(HS2_ERR_INDEX, 122);
-          src[it] = static_cast<int64_t>(valid ? pj : 0) * p.kv_tok;
-          nbytes[it] = valid ? 16u : 0u;
-          cp_async_16(kd + sw128_chunk_offset(r, chunk, 128), kg + src[it], nbytes[it]);
+          const int64_t off = static_cast<int64_t>(valid ? pj : 0) * p.kv_tok;
+          cp_async_16(kd + sw128_chunk_offset(r, chunk, 128), kg + off, valid ? 16u : 0u);
         }
         cp_async_commit();
-#pragma unroll
+#pragma unroll 4
         for (int it = 0; it < 32; ++it) {
           const int r = pw * 2 + row_sub + 4 * it;
-          cp_async_16(kd + TILE_BYTES + sw128_chunk_offset(r, chunk, 128), vg + src[it], nbytes[it]);
+          const int gi = j * 128 + r;
+          const int pj = pos_s[gi];
+          const bool valid = gi < cnt && pj >= 0 && pj < e_b;
+          const int64_t off = static_cast<int64_t>(valid ? pj : 0) * p.kv_tok;
+          cp_async_16(kd + TILE_BYTES + sw128_chunk_offset(r, chunk, 128), vg + off, valid ? 16u : 0u);
         }
         cp_async_commit();
         cp_async_wait<1>();
@@ -293,32 +339,39 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else {
     // ============================================ softmax / rescale / epilogue
-    const int r = threadIdx.x - 128;
+    const int x = (warp >= 8) ? 1 : 0;  // query tile of this warpgroup
+    const int nX = x ? nB : nA;
+    const int r = threadIdx.x - 128 - 128 * x;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    int i_row, hh;
+    const uint32_t s_tm = tmem + lane_off + x * 128;
+    const uint32_t o_tm = tmem + lane_off + 256 + x * 128;
+    int i_row, hh, i_min, diag = -1;
     if (MODE == FLASH_DENSE) {
+      const int qt = 2 * pair + x;
       i_row = qt * 128 + r;
       hh = h;
+      i_min = qt * 128;
+      diag = qt;
     } else {
+      const int mt = 2 * pair + x;
       i_row = 64 * b + mt * p.rows_tok + r / p.G;
       hh = g * p.G + r % p.G;
+      i_min = 64 * b + mt * p.rows_tok;
     }
-    const int i_min = (MODE == FLASH_DENSE) ? qt * 128 : 64 * b + mt * p.rows_tok;
+    const float sc = p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      const int buf = j & 1;
-      if (!warp_wait(&bars->s_full[buf], (j >> 1) & 1, p.limit_ns, abort_flag, 131)) {
+    for (int j = 0; j < nX; ++j) {
+      if (!warp_wait(&bars->s_full[x], j & 1, p.limit_ns, abort_flag, 131)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t s_addr = tmem + lane_off + buf * 128;
       uint32_t sr[4][32];
-      tmem_ld32(s_addr, sr[0]);
-      tmem_ld32(s_addr + 32, sr[1]);
-      tmem_ld32(s_addr + 64, sr[2]);
-      tmem_ld32(s_addr + 96, sr[3]);
+      tmem_ld32(s_tm, sr[0]);
+      tmem_ld32(s_tm + 32, sr[1]);
+      tmem_ld32(s_tm + 64, sr[2]);
+      tmem_ld32(s_tm + 96, sr[3]);
       tmem_ld_wait();
       reg_fence(sr[0]);
       reg_fence(sr[1]);
@@ -327,7 +380,7 @@ __global__ void __launch_bounds__(256, 1)
       // ---- mask
       bool need_mask;
       if (MODE == FLASH_DENSE) {
-        need_mask = (j == qt);
+        need_mask = (j == diag);
       } else {
         const int last = j * 128 + 127;
         need_mask = (last >= cnt) || (pos_s[last] > i_min);
@@ -352,10 +405,19 @@ __global__ void __launch_bounds__(256, 1)
           }
         }
       }
-      float mx = -INFINITY;
+      // ---- row max: 8 independent partial maxima
+      float mx8[8];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c >> 5][c & 31]));
-      const float m_new = fmaxf(m_used, mx * p.scale_log2);
+      for (int q = 0; q < 8; ++q) mx8[q] = __uint_as_float(sr[q >> 1][(q & 1) * 16]);
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        if ((c & 15) == 0) continue;
+        const int q = c >> 4;
+        mx8[q] = fmaxf(mx8[q], __uint_as_float(sr[c >> 5][c & 31]));
+      }
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float m_new = fmaxf(m_used, mx * sc);
       float alpha = 1.f;
       const bool resc = m_new > m_used + 8.f;
       if (resc) {
@@ -364,55 +426,66 @@ __global__ void __launch_bounds__(256, 1)
       }
       const float mu = (m_used == -INFINITY) ? 0.f : m_used;
       l *= alpha;
-      // ---- P = exp2(s * scale - m), into TMEM over S
-      float rs = 0.f;
+      // ---- P = exp2(s * scale - m) into TMEM over S; on unmasked tiles the
+      // last 32 columns go through the FMA pipes
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
+        if (c == 3 && !need_mask) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), p.scale_log2, -mu));
-          const float bb = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), p.scale_log2, -mu));
-          rs += a + bb;
-          pk[e] = pack_bf16x2(a, bb);
+          for (int e = 0; e < 16; ++e) {
+            const float e0 = exp2_fma3(fmaf(__uint_as_float(sr[c][2 * e]), sc, -mu));
+            const float e1 = exp2_fma3(fmaf(__uint_as_float(sr[c][2 * e + 1]), sc, -mu));
+            rs4[e & 3] += e0 + e1;
+            pk[e] = pack_bf16x2(e0, e1);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float e0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sc, -mu));
+            const float e1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sc, -mu));
+            rs4[e & 3] += e0 + e1;
+            pk[e] = pack_bf16x2(e0, e1);
+          }
         }
-        tmem_st16(s_addr + c * 16, pk);
+        tmem_st16(s_tm + c * 16, pk);
       }
-      l += rs;
-      // ---- O rescale (needs PV_{j-1} complete)
+      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      // ---- O rescale (needs PV(j-1) complete)
       if (j > 0) {
-        if (!warp_wait(&bars->o_done, (j - 1) & 1, p.limit_ns, abort_flag, 132)) {
+        if (!warp_wait(&bars->o_done[x], (j - 1) & 1, p.limit_ns, abort_flag, 132)) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll
+#pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t orr[32];
-            tmem_ld32(tmem + lane_off + 256 + c * 32, orr);
+            tmem_ld32(o_tm + c * 32, orr);
             tmem_ld_wait();
             reg_fence(orr);
 #pragma unroll
             for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-            tmem_st32(tmem + lane_off + 256 + c * 32, orr);
+            tmem_st32(o_tm + c * 32, orr);
           }
         }
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_ready);
+      mbar_arrive(&bars->p_ready[x]);
     }
     // ---- epilogue
-    const bool row_live = i_row < p.L;  // a last dense tile may hang past L
-    if (ok && ntiles > 0 && warp_wait(&bars->o_done, (ntiles - 1) & 1, p.limit_ns, abort_flag, 133)) {
+    const bool row_live = i_row < p.L && (x == 0 || has_b);  // a last dense tile may hang past L
+    __nv_bfloat16* orow = p.o + static_cast<int64_t>(i_row) * p.o_tok + static_cast<int64_t>(hh) * p.o_head;
+    if (ok && nX > 0 && warp_wait(&bars->o_done[x], (nX - 1) & 1, p.limit_ns, abort_flag, 133)) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = p.o + static_cast<int64_t>(i_row) * p.o_tok + static_cast<int64_t>(hh) * p.o_head;
-#pragma unroll
+#pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t orr[32];
-        tmem_ld32(tmem + lane_off + 256 + c * 32, orr);
+        tmem_ld32(o_tm + c * 32, orr);
         tmem_ld_wait();
         reg_fence(orr);
         uint32_t pk[16];
@@ -426,11 +499,10 @@ __global__ void __launch_bounds__(256, 1)
             dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
       }
-      if (MODE == FLASH_DENSE && row_live) {
+      if (MODE == FLASH_DENSE && row_live)
         p.lse[static_cast<int64_t>(hh) * p.L + i_row] = (m_used + log2f(l)) * 0.69314718055994530942f;
-      }
-    } else if (ntiles == 0 && MODE == FLASH_SPARSE) {
-      __nv_bfloat16* orow = p.o + static_cast<int64_t>(i_row) * p.o_tok + static_cast<int64_t>(hh) * p.o_head;
+    } else if (MODE == FLASH_SPARSE && ok && n == 0 && row_live) {
+      // an empty list: the rows attend to nothing
       uint4* dst = reinterpret_cast<uint4*>(orow);
       for (int v4 = 0; v4 < 16; ++v4) dst[v4] = make_uint4(0, 0, 0, 0);
     }

@@ -130,6 +130,7 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
   p.Hkv = s->Hkv;
   p.G = s->Hq / s->Hkv;
   p.nqt = s->L / 128 + (s->L % 128 ? 1 : 0);
+  p.npairs = (p.nqt + 1) / 2;
   p.scale_log2 = scale_log2(s->d);
   p.o = static_cast<__nv_bfloat16*>(o);
   p.o_tok = s->q_tok_stride;
@@ -139,8 +140,8 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
   p.flags = g_flags;
   static int attr = set_smem(flash_fwd_kernel<FLASH_DENSE>, FL_SMEM_DENSE);
   if (attr) return attr;
-  const unsigned grid = static_cast<unsigned>(p.nqt * s->Hq);
-  flash_fwd_kernel<FLASH_DENSE><<<grid, 256, FL_SMEM_DENSE, st>>>(mq, mk, mv, p);
+  const unsigned grid = static_cast<unsigned>(p.npairs * s->Hq);
+  flash_fwd_kernel<FLASH_DENSE><<<grid, FL_THREADS, FL_SMEM_DENSE, st>>>(mq, mk, mv, p);
   return launched();
 }
 
@@ -159,6 +160,7 @@ int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* 
   p.nb = s->L / 64;
   p.list_len = s->topk + s->recent;
   p.mtiles = (64 * G) / 128;
+  p.mpairs = (p.mtiles + 1) / 2;
   p.rows_tok = rows_tok;
   p.scale_log2 = scale_log2(s->d);
   p.k = static_cast<const __nv_bfloat16*>(k);
@@ -174,8 +176,8 @@ int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* 
   p.flags = g_flags;
   static int attr = set_smem(flash_fwd_kernel<FLASH_SPARSE>, FL_SMEM_SPARSE);
   if (attr) return attr;
-  const unsigned grid = static_cast<unsigned>(p.nb * s->Hkv * p.mtiles);
-  flash_fwd_kernel<FLASH_SPARSE><<<grid, 256, FL_SMEM_SPARSE, st>>>(mq, mq, mq, p);
+  const unsigned grid = static_cast<unsigned>(p.nb * s->Hkv * p.mpairs);
+  flash_fwd_kernel<FLASH_SPARSE><<<grid, FL_THREADS, FL_SMEM_SPARSE, st>>>(mq, mq, mq, p);
   return launched();
 }
 
@@ -186,7 +188,7 @@ int launch_importance_g(const CUtensorMap& mq, const CUtensorMap& mk, const ImpP
                         cudaStream_t st) {
   static int attr = set_smem(importance_kernel<G>, imp_smem_bytes(G));
   if (attr) return attr;
-  importance_kernel<G><<<grid, 256, imp_smem_bytes(G), st>>>(mq, mk, p);
+  importance_kernel<G><<<grid, IMP_THREADS, imp_smem_bytes(G), st>>>(mq, mk, p);
   return launched();
 }
 
@@ -240,6 +242,16 @@ int launch_select(const hs2_shape* s, const float* imp, int64_t row_stride, int 
   p.cnt = cnt;
   topk_select_kernel<<<static_cast<unsigned>(s->Hkv * (b1 - b0)), SEL_THREADS, 0, st>>>(p);
   return launched();
+}
+
+__global__ void exp2_check_kernel(const float* x, float* y0, float* y3, float* y4, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = x[i];
+    y0[i] = ex2_approx(v);
+    y3[i] = exp2_fma3(v);
+    y4[i] = exp2_fma4(v);
+  }
 }
 
 int64_t strip_stride(const hs2_shape* s, int b_last) {
@@ -305,6 +317,14 @@ const char* hs2_strerror(int code) {
 }
 
 int hs2_version(void) { return 100; }
+
+int hs2_exp2_check(const float* x, float* y_mufu, float* y_fma3, float* y_fma4, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y_mufu || !y_fma3 || !y_fma4))) return HS2_ERR_INVALID_ARG;
+  if (n == 0) return HS2_OK;
+  const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096));
+  exp2_check_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_mufu, y_fma3, y_fma4, n);
+  return launched();
+}
 
 uint64_t hs2_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 

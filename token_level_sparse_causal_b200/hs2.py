@@ -21,7 +21,7 @@ HS2_KV_BF16, HS2_KV_E4M3 = 0, 1
 
 EXPORTS = ("hs2_full_attn_select", "hs2_sparse_attn", "hs2_sync", "hs2_attn_fwd", "hs2_importance",
            "hs2_topk_select", "hs2_strerror", "hs2_debug_set", "hs2_version", "hs2_launch_count",
-           "hs2_full_attn_select_static")
+           "hs2_full_attn_select_static", "hs2_exp2_check")
 
 
 class Hs2Shape(ctypes.Structure):
@@ -50,6 +50,7 @@ _SIGS = {
     "hs2_importance": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i64, _vp],
     "hs2_topk_select": [ctypes.POINTER(Hs2Shape), _vp, _i64, _i32, _i32, _vp, _vp, _vp],
     "hs2_debug_set": [_u64, _u32],
+    "hs2_exp2_check": [_vp, _vp, _vp, _vp, _i64, _vp],
     "hs2_version": [],
 }
 
@@ -149,6 +150,11 @@ def hs2_sync(stream=None) -> None:
 
 def hs2_launch_count() -> int:
     return int(lib().hs2_launch_count())
+
+
+def hs2_exp2_check(x, y_mufu, y_fma3, y_fma4, stream=None) -> None:
+    _check(lib().hs2_exp2_check(_ptr(x), _ptr(y_mufu), _ptr(y_fma3), _ptr(y_fma4), x.numel(), _stream(stream)),
+           "hs2_exp2_check")
 
 
 def hs2_debug_set(wait_limit_ns: int = 2_000_000_000, flags: int = 0) -> None:
