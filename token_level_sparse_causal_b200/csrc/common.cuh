@@ -80,6 +80,66 @@ __device__ __forceinline__ float exp2_fma4(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// ---- packed fp32 pairs (sm_100 executes f32x2 FMA/ADD as one instruction)
+
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2_fma3 / exp2_fma4 on a pair, with the arithmetic in f32x2 form.
+template <int DEG>
+__device__ __forceinline__ uint64_t exp2_fma_x2(uint64_t xv) {
+  float a, b;
+  f2_unpack(xv, a, b);
+  const uint64_t x = f2_pack(fmaxf(a, -125.0f), fmaxf(b, -125.0f));
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(x, magic);
+  const uint64_t tm = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = f2_fma(tm, f2_pack(-1.0f, -1.0f), x);
+  uint64_t p;
+  if (DEG == 3) {
+    p = f2_fma(f2_pack(EXP2_D3_C3, EXP2_D3_C3), f, f2_pack(EXP2_D3_C2, EXP2_D3_C2));
+    p = f2_fma(p, f, f2_pack(EXP2_D3_C1, EXP2_D3_C1));
+    p = f2_fma(p, f, f2_pack(EXP2_D3_C0, EXP2_D3_C0));
+  } else {
+    p = f2_fma(f2_pack(EXP2_D4_C4, EXP2_D4_C4), f, f2_pack(EXP2_D4_C3, EXP2_D4_C3));
+    p = f2_fma(p, f, f2_pack(EXP2_D4_C2, EXP2_D4_C2));
+    p = f2_fma(p, f, f2_pack(EXP2_D4_C1, EXP2_D4_C1));
+    p = f2_fma(p, f, f2_pack(EXP2_D4_C0, EXP2_D4_C0));
+  }
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
+}
+
+__device__ __forceinline__ uint64_t ex2_x2(uint64_t xv) {
+  float a, b;
+  f2_unpack(xv, a, b);
+  return f2_pack(ex2_approx(a), ex2_approx(b));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

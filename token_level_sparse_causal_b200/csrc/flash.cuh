@@ -34,10 +34,10 @@
 //
 // Softmax runs in the log2 domain with a lazily updated reference max: O is
 // rescaled only when a row max grows by more than 8 (P stays below 256; the
-// final O / l is exact up to rounding).  A quarter of the exponentials of
-// every unmasked tile are computed on the FMA pipes (exp2_fma3) so the MUFU
-// unit stops being the bottleneck; row max and row sum use independent
-// partial accumulators.
+// final O / l is exact up to rounding).  Arguments and row sums use packed
+// f32x2 FMA/ADD and the row max 3-input max, in independent partial chains:
+// the softmax is bound by instruction issue, not by the MUFU exponential
+// unit (moving exponentials to FMA-pipe polynomials measured slower).
 #pragma once
 
 #include "common.cuh"
@@ -405,18 +405,18 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           }
         }
       }
-      // ---- row max: 8 independent partial maxima
-      float mx8[8];
+      // ---- row max: 4 independent chains of 3-input max
+      float mx4[4];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) mx8[q] = __uint_as_float(sr[q >> 1][(q & 1) * 16]);
+      for (int q = 0; q < 4; ++q) mx4[q] = __uint_as_float(sr[q][0]);
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        if ((c & 15) == 0) continue;
-        const int q = c >> 4;
-        mx8[q] = fmaxf(mx8[q], __uint_as_float(sr[c >> 5][c & 31]));
+      for (int q = 0; q < 4; ++q) {
+#pragma unroll
+        for (int e = 0; e < 15; ++e)
+          mx4[q] = fmax3(mx4[q], __uint_as_float(sr[q][1 + 2 * e]), __uint_as_float(sr[q][2 + 2 * e]));
+        mx4[q] = fmaxf(mx4[q], __uint_as_float(sr[q][31]));
       }
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
       const float m_new = fmaxf(m_used, mx * sc);
       float alpha = 1.f;
       const bool resc = m_new > m_used + 8.f;
@@ -426,32 +426,31 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       }
       const float mu = (m_used == -INFINITY) ? 0.f : m_used;
       l *= alpha;
-      // ---- P = exp2(s * scale - m) into TMEM over S; on unmasked tiles the
-      // last 32 columns go through the FMA pipes
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      // ---- P = exp2(s * scale - m) into TMEM over S (arguments and row sums
+      // as packed f32x2)
+      const uint64_t sc2 = f2_pack(sc, sc), nmu2 = f2_pack(-mu, -mu);
+      uint64_t sum2[2] = {0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
-        if (c == 3 && !need_mask) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float e0 = exp2_fma3(fmaf(__uint_as_float(sr[c][2 * e]), sc, -mu));
-            const float e1 = exp2_fma3(fmaf(__uint_as_float(sr[c][2 * e + 1]), sc, -mu));
-            rs4[e & 3] += e0 + e1;
-            pk[e] = pack_bf16x2(e0, e1);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float e0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sc, -mu));
-            const float e1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sc, -mu));
-            rs4[e & 3] += e0 + e1;
-            pk[e] = pack_bf16x2(e0, e1);
-          }
+        for (int e = 0; e < 16; ++e) {
+          const uint64_t a2 =
+              f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])), sc2, nmu2);
+          const uint64_t p2 = ex2_x2(a2);
+          sum2[e & 1] = f2_add(sum2[e & 1], p2);
+          float e0, e1;
+          f2_unpack(p2, e0, e1);
+          pk[e] = pack_bf16x2(e0, e1);
         }
         tmem_st16(s_tm + c * 16, pk);
       }
-      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(sum2[0], a0, a1);
+        f2_unpack(sum2[1], b0, b1);
+        l += (a0 + a1) + (b0 + b1);
+      }
       // ---- O rescale (needs PV(j-1) complete)
       if (j > 0) {
         if (!warp_wait(&bars->o_done[x], (j - 1) & 1, p.limit_ns, abort_flag, 132)) {

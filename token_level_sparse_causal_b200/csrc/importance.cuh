@@ -16,12 +16,14 @@
 // columns are split in sub-tiles of N = min(256, 64G); two TMEM buffers let
 // the tensor core fill one sub-tile while the epilogue drains the other.
 //
-// CTA = 12 warps: warp 0 TMA (Q block once, then K tiles), warp 1 MMA issue
-// and TMEM owner, warps 4-7 and 8-11 two epilogue warpgroups that split the
-// columns of each sub-tile (thread r of both <-> key r of the tile); the
-// second group hands its partial sums to the first through shared memory.
-// Of every 8 columns, 3 take their exponential on the FMA pipes (exp2_fma4,
-// relative error 2.6e-6) and 5 on the MUFU unit, which balances the two.
+// CTA = 20 warps: warp 0 TMA (Q block once, then K tiles), warp 1 MMA issue
+// and TMEM owner, warps 4-19 four epilogue warpgroups that split the columns
+// of each sub-tile in quarters (thread r of every group <-> key r of the
+// tile).  Each thread issues all of its TMEM loads for a sub-tile before one
+// wait, and groups 2-4 hand their partial sums to group 1 through shared
+// memory, which adds them in a fixed order (the result is deterministic, so
+// hs2_importance reproduces exactly what the selection saw).  Arguments and
+// sums use packed f32x2 FMA/ADD; the exponentials run on the MUFU unit.
 // Work item = (KV head, block, chunk of IMP_CK keys); the grid is
 // (chunks of the longest row of the strip) x (Hkv * blocks).
 #pragma once
@@ -32,7 +34,7 @@
 namespace hs2 {
 
 constexpr int IMP_CK = 2048;   // keys per CTA
-constexpr int IMP_STAGES = 2;  // K tile ring
+constexpr int IMP_STAGES = 2;  // K tile ring (deeper rings measured no faster)
 
 struct ImpParams {
   int L, Hq, Hkv, G, recent, b0, nbs;
@@ -63,8 +65,11 @@ __host__ __device__ constexpr uint32_t imp_kv_off(int G) { return imp_q_bytes(G)
 __host__ __device__ constexpr uint32_t imp_bar_off(int G) { return imp_q_bytes(G) + IMP_STAGES * TILE_BYTES; }
 __host__ __device__ constexpr uint32_t imp_lse_off(int G) { return imp_bar_off(G) + 256; }
 __host__ __device__ constexpr uint32_t imp_part_off(int G) { return imp_lse_off(G) + static_cast<uint32_t>(64 * G) * 4u; }
-__host__ __device__ constexpr uint32_t imp_smem_bytes(int G) { return imp_part_off(G) + 2u * 128u * 4u + 1024u; }
-constexpr int IMP_THREADS = 384;
+constexpr int IMP_GROUPS = 4;  // epilogue warpgroups
+constexpr int IMP_THREADS = 128 + 128 * IMP_GROUPS;
+__host__ __device__ constexpr uint32_t imp_smem_bytes(int G) {
+  return imp_part_off(G) + (IMP_GROUPS - 1) * 2u * 128u * 4u + 1024u;
+}
 
 template <int G>
 __global__ void __launch_bounds__(IMP_THREADS, 1)
@@ -90,7 +95,7 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
   uint8_t* smem = align1024(smem_raw);
   ImpBars* bars = reinterpret_cast<ImpBars*>(smem + imp_bar_off(G));
   float* nlse = reinterpret_cast<float*>(smem + imp_lse_off(G));
-  float* part = reinterpret_cast<float*>(smem + imp_part_off(G));  // [2][128] partial sums of group 2
+  float* part = reinterpret_cast<float*>(smem + imp_part_off(G));  // [groups-1][2][128] partial sums
   const uint32_t q_base = smem_u32(smem);
   const uint32_t k_base = smem_u32(smem + imp_kv_off(G));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -104,8 +109,8 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->acc_full[s], 1);
-      mbar_init(&bars->acc_empty[s], 256);
-      mbar_init(&bars->part_full[s], 128);
+      mbar_init(&bars->acc_empty[s], 128 * IMP_GROUPS);
+      mbar_init(&bars->part_full[s], 128 * (IMP_GROUPS - 1));
       mbar_init(&bars->part_empty[s], 128);
     }
     mbar_init(&bars->fin, 1);
@@ -185,16 +190,17 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
       wait_done(&bars->fin, 0, p.limit_ns, 214);
     }
   } else if (warp >= 4) {
-    const int grp = (warp >= 8) ? 1 : 0;        // which half of each sub-tile's columns
+    const int grp = (warp - 4) >> 2;              // epilogue group 0..IMP_GROUPS-1
     const int r = threadIdx.x - 128 - 128 * grp;  // key row of the tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    constexpr int HALF = NSUB / 2;                // columns per group and sub-tile
+    constexpr int QCOLS = NSUB / IMP_GROUPS;      // columns per group and sub-tile (32 or 64)
+    constexpr int NLD = QCOLS / 32;
     float* out = p.imp + (static_cast<int64_t>(g) * p.nbs + (b - p.b0)) * p.row_stride;
-    const float c2 = p.scale_log2;
+    const uint64_t c2p = f2_pack(p.scale_log2, p.scale_log2);
     int u = 0;
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      uint64_t acc2[2] = {0ull, 0ull};
       for (int sub = 0; sub < SUBS; ++sub, ++u) {
         const int buf = u & 1;
         if (!warp_wait(&bars->acc_full[buf], (u >> 1) & 1, p.limit_ns, abort_flag, 221)) {
@@ -202,59 +208,58 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
           break;
         }
         tc_fence_after();
-        const int col0 = grp * HALF;
+        const int col0 = grp * QCOLS;
+        uint32_t sr[NLD][32];
+#pragma unroll
+        for (int c = 0; c < NLD; ++c) tmem_ld32(tmem + lane_off + buf * NSUB + col0 + c * 32, sr[c]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < NLD; ++c) reg_fence(sr[c]);
+        tc_fence_before();
+        mbar_arrive(&bars->acc_empty[buf]);  // the buffer's data is in registers now
         const float4* nl4 = reinterpret_cast<const float4*>(nlse + sub * NSUB + col0);
-#pragma unroll 1
-        for (int c = 0; c < HALF / 32; ++c) {
-          uint32_t sr[32];
-          tmem_ld32(tmem + lane_off + buf * NSUB + col0 + c * 32, sr);
-          tmem_ld_wait();
-          reg_fence(sr);
+#pragma unroll
+        for (int c = 0; c < NLD; ++c) {
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
             const float4 nl = nl4[c * 8 + e4];  // broadcast read
-            const float a0 = fmaf(__uint_as_float(sr[4 * e4 + 0]), c2, nl.x);
-            const float a1 = fmaf(__uint_as_float(sr[4 * e4 + 1]), c2, nl.y);
-            const float a2 = fmaf(__uint_as_float(sr[4 * e4 + 2]), c2, nl.z);
-            const float a3 = fmaf(__uint_as_float(sr[4 * e4 + 3]), c2, nl.w);
-            if ((e4 & 1) == 0) {  // 3 of every 8 columns on the FMA pipes
-              acc[0] += exp2_fma4(a0);
-              acc[1] += exp2_fma4(a1);
-              acc[2] += ex2_approx(a2);
-              acc[3] += ex2_approx(a3);
-            } else {
-              acc[0] += exp2_fma4(a0);
-              acc[1] += ex2_approx(a1);
-              acc[2] += ex2_approx(a2);
-              acc[3] += ex2_approx(a3);
-            }
+            const uint64_t a01 = f2_fma(f2_pack(__uint_as_float(sr[c][4 * e4]), __uint_as_float(sr[c][4 * e4 + 1])),
+                                        c2p, f2_pack(nl.x, nl.y));
+            const uint64_t a23 = f2_fma(
+                f2_pack(__uint_as_float(sr[c][4 * e4 + 2]), __uint_as_float(sr[c][4 * e4 + 3])), c2p,
+                f2_pack(nl.z, nl.w));
+            acc2[0] = f2_add(acc2[0], ex2_x2(a01));
+            acc2[1] = f2_add(acc2[1], ex2_x2(a23));
           }
         }
-        tc_fence_before();
-        mbar_arrive(&bars->acc_empty[buf]);
       }
       if (!ok) break;
-      // Hand group 2's partial sums to group 1 through a double-buffered
-      // shared array guarded by mbarriers (bounded waits: no CTA barrier
-      // inside the loop, so an aborted role can never strand the others).
-      const float mine = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      // Groups 2..IMP_GROUPS hand their partial sums to group 1 through a
+      // double-buffered shared array guarded by mbarriers (bounded waits: no
+      // CTA barrier inside the loop, so an aborted role never strands others).
+      float m0, m1, m2, m3;
+      f2_unpack(acc2[0], m0, m1);
+      f2_unpack(acc2[1], m2, m3);
+      const float mine = (m0 + m1) + (m2 + m3);
       const int pb = t & 1;
-      if (grp == 1) {
+      if (grp > 0) {
         if (t >= 2 && !mbar_wait(&bars->part_empty[pb], ((t >> 1) - 1) & 1, p.limit_ns, abort_flag, 222)) {
           ok = false;
           break;
         }
-        part[pb * 128 + r] = mine;
+        part[((grp - 1) * 2 + pb) * 128 + r] = mine;
         mbar_arrive(&bars->part_full[pb]);
       } else {
         if (!mbar_wait(&bars->part_full[pb], (t >> 1) & 1, p.limit_ns, abort_flag, 223)) {
           ok = false;
           break;
         }
-        const float other = part[pb * 128 + r];
+        float total = mine;
+#pragma unroll
+        for (int q = 0; q < IMP_GROUPS - 1; ++q) total += part[(q * 2 + pb) * 128 + r];
         mbar_arrive(&bars->part_empty[pb]);
         const int j = j0 + t * 128 + r;
-        if (j < n_c) out[j] = mine + other;
+        if (j < n_c) out[j] = total;
       }
     }
   }
