@@ -34,23 +34,38 @@ def guards_intact(base):
     return bool((base[:GUARD] == s).all() and (base[-GUARD:] == s).all())
 
 
+def decode_kv(t, scale):
+    """fp64 K or V from the exact stored bytes (bf16, or e4m3 codes x scale)."""
+    if scale is None:
+        return orc.decode_bf16(inputs.as_u16(t))
+    return orc.dequantize(inputs.as_u8(t), scale.detach().cpu().numpy())
+
+
 def decode(x):
     """fp64 oracle inputs from the exact bytes the GPU reads."""
     out = {"Q": [orc.decode_bf16(inputs.as_u16(q)) for q in x["q_layers"]]}
-    out["K"] = orc.decode_bf16(inputs.as_u16(x["k"]))
-    out["V"] = orc.decode_bf16(inputs.as_u16(x["v"]))
+    out["K"] = decode_kv(x["k"], x.get("k_scale"))
+    out["V"] = decode_kv(x["v"], x.get("v_scale"))
     return out
 
 
 def to_dev(x, dev):
-    return {"q_layers": [q.to(dev) for q in x["q_layers"]], "k": x["k"].to(dev), "v": x["v"].to(dev)}
+    mv = lambda t: None if t is None else t.to(dev)
+    return {"q_layers": [q.to(dev) for q in x["q_layers"]], "k": x["k"].to(dev), "v": x["v"].to(dev),
+            "k_scale": mv(x.get("k_scale")), "v_scale": mv(x.get("v_scale"))}
+
+
+def shape_of(wl, xd):
+    kvd = hs2.HS2_KV_E4M3 if xd["k"].dtype == torch.uint8 else hs2.HS2_KV_BF16
+    return hs2.make_shape(xd["q_layers"][0], xd["k"], wl.topk, wl.recent, kv_dtype=kvd)
 
 
 def run_path(wl, xd, stream=None, guards=False):
     """Full layer + every sparse layer through the C ABI; returns tensors."""
     q0, k, v = xd["q_layers"][0], xd["k"], xd["v"]
+    ks, vs = xd.get("k_scale"), xd.get("v_scale")
     dev = q0.device
-    shape = hs2.make_shape(q0, k, wl.topk, wl.recent)
+    shape = shape_of(wl, xd)
     nb = wl.L // wl.block
     res = {"shape": shape, "bases": []}
     if guards:
@@ -64,7 +79,7 @@ def run_path(wl, xd, stream=None, guards=False):
         idx = torch.empty((wl.Hkv, nb, wl.topk + wl.recent), device=dev, dtype=torch.int32)
         cnt = torch.empty((wl.Hkv, nb), device=dev, dtype=torch.int32)
     ws = torch.empty(hs2.workspace_bytes(shape) // 4 + 4, device=dev, dtype=torch.float32)
-    hs2.hs2_full_attn_select(shape, q0, k, v, None, None, o, lse, idx, cnt, ws, stream)
+    hs2.hs2_full_attn_select(shape, q0, k, v, ks, vs, o, lse, idx, cnt, ws, stream)
     sparse = []
     for ql in xd["q_layers"][1:]:
         if guards:
@@ -72,7 +87,7 @@ def run_path(wl, xd, stream=None, guards=False):
             res["bases"].append(olb)
         else:
             ol = torch.empty_like(ql)
-        hs2.hs2_sparse_attn(shape, ql, k, v, None, None, idx, cnt, ol, stream)
+        hs2.hs2_sparse_attn(shape, ql, k, v, ks, vs, idx, cnt, ol, stream)
         sparse.append(ol)
     hs2.hs2_sync(stream)
     res.update(o=o, lse=lse, idx=idx, cnt=cnt, sparse=sparse)
@@ -84,7 +99,7 @@ def gpu_importance(shape, xd, lse, b0, b1):
     L, recent = shape.L, shape.recent
     stride = max(4, ((max(0, min(L, 64 * b1) - recent) + 3) // 4) * 4)
     imp = torch.full((shape.Hkv, b1 - b0, stride), float("nan"), device=lse.device, dtype=torch.float32)
-    hs2.hs2_importance(shape, xd["q_layers"][0], xd["k"], None, lse, b0, b1, imp, stride)
+    hs2.hs2_importance(shape, xd["q_layers"][0], xd["k"], xd.get("k_scale"), lse, b0, b1, imp, stride)
     hs2.hs2_sync()
     return imp
 

@@ -250,6 +250,7 @@ class _Rows:
 def _sampled_check(wl, blocks, groups):
     xd = inputs.make_inputs(wl, device=DEV)
     r = H.run_path(wl, xd)
+    fp8 = xd.get("k_scale") is not None
     G = wl.G
     for b in blocks:
         s_b, e_b = orc.block_rows(b, wl.L, 64)
@@ -257,8 +258,8 @@ def _sampled_check(wl, blocks, groups):
         for g in groups:
             hs = slice(g * G, (g + 1) * G)
             Qb = [_Rows(orc.decode_bf16(inputs.as_u16(q[s_b:e_b, hs])), s_b, wl.L) for q in xd["q_layers"]]
-            K = orc.decode_bf16(inputs.as_u16(xd["k"][:e_b, g:g + 1]))
-            V = orc.decode_bf16(inputs.as_u16(xd["v"][:e_b, g:g + 1]))
+            K = H.decode_kv(xd["k"][:e_b, g:g + 1], xd["k_scale"][:e_b, g:g + 1] if fp8 else None)
+            V = H.decode_kv(xd["v"][:e_b, g:g + 1], xd["v_scale"][:e_b, g:g + 1] if fp8 else None)
             O, LSE = orc.dense_attn(Qb[0], K, V, s_b, e_b)
             H.bf16_close(r["o"][s_b:e_b, hs].float().cpu().numpy(), O, f"O b{b} g{g}")
             assert np.abs(r["lse"][hs, s_b:e_b].cpu().numpy() - LSE).max() <= H.LSE_ATOL
@@ -291,6 +292,75 @@ def test_full_size_128k_workload_sampled():
     blocks = [18, wl.nb - 1] + [int(b) for b in rng.integers(19, wl.nb - 1, 2)]
     _sampled_check(wl, blocks, groups=[3, 7])
     torch.cuda.empty_cache()
+
+
+def test_full_size_256k_chain_workload_sampled():
+    wl = inputs.WORKLOADS["c4"]
+    rng = np.random.default_rng(3)
+    blocks = [18, wl.nb - 1, int(rng.integers(19, wl.nb - 1))]
+    _sampled_check(wl, blocks, groups=[1])
+    torch.cuda.empty_cache()
+
+
+def test_full_size_1m_fp8_workload_sampled():
+    """L = 1M with an e4m3 K/V cache and per-token scales."""
+    wl = inputs.WORKLOADS["c5"]
+    rng = np.random.default_rng(4)
+    blocks = [18, wl.nb - 1, int(rng.integers(19, wl.nb - 1))]
+    _sampled_check(wl, blocks, groups=[2])
+    torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------ FP8 (e4m3) cache --
+
+def _fp8_wl(L, Hq, Hkv, n_sparse=1, seed=31, topk=1024):
+    return inputs.Workload(f"f{L}_{Hq}x{Hkv}", L, Hq, Hkv, n_sparse, seed, kv_dtype="e4m3", topk=topk)
+
+
+@pytest.mark.parametrize("L,Hq,Hkv", [(1088, 8, 1), (640, 8, 2), (512, 4, 2)])
+def test_fp8_attn_fwd_matches_oracle(L, Hq, Hkv):
+    wl = _fp8_wl(L, Hq, Hkv)
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    shape = H.shape_of(wl, xd)
+    o, ob = H.guarded((L, Hq, 128), torch.bfloat16, DEV)
+    lse, lb = H.guarded((Hq, L), torch.float32, DEV)
+    hs2.hs2_attn_fwd(shape, xd["q_layers"][0], xd["k"], xd["v"], xd["k_scale"], xd["v_scale"], o, lse)
+    hs2.hs2_sync()
+    D = H.decode(x)
+    O, LSE = orc.dense_attn(D["Q"][0], D["K"], D["V"])
+    H.bf16_close(o.float().cpu().numpy(), O, "O (fp8 cache)")
+    assert np.abs(lse.cpu().numpy() - LSE).max() <= H.LSE_ATOL
+    assert H.guards_intact(ob) and H.guards_intact(lb)
+
+
+@pytest.mark.parametrize("L,Hq,Hkv", [(2304, 8, 1), (1536, 4, 2)])
+def test_fp8_importance_select_and_sparse_match_oracle(L, Hq, Hkv):
+    wl = _fp8_wl(L, Hq, Hkv, n_sparse=1, topk=1000)
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    r = H.run_path(wl, xd, guards=True)
+    nb = L // 64
+    imp = H.gpu_importance(r["shape"], xd, r["lse"], 0, nb).cpu().numpy().astype(np.float64)
+    D = H.decode(x)
+    _, LSE = orc.dense_attn(D["Q"][0], D["K"], D["V"])
+    idx, cnt = r["idx"].cpu().numpy(), r["cnt"].cpu().numpy()
+    G = wl.G
+    ref_sp = np.empty((L, Hq, 128))
+    worst = 0.0
+    for b in range(nb):
+        s_b, e_b = orc.block_rows(b, L, 64)
+        for g in range(Hkv):
+            ref = orc.importance(D["Q"][0], D["K"], LSE[:, s_b:e_b], b, g, 64, 128)
+            got = imp[g, b, :ref.size]
+            if ref.size:
+                worst = max(worst, (np.abs(got - ref) / np.maximum(np.abs(ref), 1e-30)).max())
+            want, wc = orc.select(got, wl.topk, 128, e_b)
+            assert cnt[g, b] == wc and np.array_equal(idx[g, b], want), (g, b)
+            ref_sp[s_b:e_b, g * G:(g + 1) * G] = orc.sparse_attn(D["Q"][1], D["K"], D["V"], idx[g, b], wc, b, g, 64)
+    assert worst <= H.IMP_RTOL, worst
+    H.bf16_close(r["sparse"][0].float().cpu().numpy(), ref_sp, "sparse (fp8 cache)")
+    assert all(H.guards_intact(bb) for bb in r["bases"])
 
 
 # -------------------------------------------------- device-side failures --

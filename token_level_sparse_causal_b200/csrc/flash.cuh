@@ -19,9 +19,17 @@
 // CTA = 12 warps:
 //   warp 0      TMA: Q tiles (both modes), K/V tiles (dense)
 //   warp 1      TMEM allocation; one thread issues every tcgen05.mma
-//   warps 2-3   K/V gather (sparse)
+//   warps 2-3   K/V gather (sparse, bf16 cache); with an FP8 cache: convert Q
+//               to f16 in place, then load, convert and scale every K/V tile
 //   warps 4-7   softmax / rescale / epilogue of query tile A (thread r <-> row r)
 //   warps 8-11  the same for query tile B
+//
+// FP8 e4m3 cache (KV8): every e4m3 value is an f16 value, so codes are
+// converted exactly to f16 (one cvt per pair), Q is converted bf16 -> f16 in
+// shared memory after its TMA load, and all MMAs run kind::f16 on f16
+// operands.  The per-token K scale (times log2(e)/sqrt(d)) multiplies the S
+// columns in fp32; the V scale is folded into the converted V rows.
+// (HySparse2 architecture summary, cost paragraph: FP8 KV cache.)
 //
 // Tensor memory (512 columns): S_A [0,128), S_B [128,256), O_A [256,384),
 // O_B [384,512).  P (bf16) is written over the first 64 columns of its S and
@@ -51,6 +59,8 @@ constexpr uint32_t TILE_BYTES = 128u * 128u * 2u;  // one 128 x 128 bf16 tile
 constexpr uint32_t HALF_BYTES = 128u * 64u * 2u;   // its d-half (128 rows x 128 B)
 constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
+constexpr uint32_t IDESC_S_F16 = idesc_f16_f32(128, 128, 0, 0);
+constexpr uint32_t IDESC_PV_F16 = idesc_f16_f32(128, 128, 0, 1);
 constexpr int FLASH_DENSE = 0;
 constexpr int FLASH_SPARSE = 1;
 constexpr uint32_t FLAG_SKIP_LOADS = 1u;
@@ -63,6 +73,10 @@ struct FlashParams {
   float scale_log2;                    // log2(e) / sqrt(d)
   const __nv_bfloat16* k;              // gather sources (sparse)
   const __nv_bfloat16* v;
+  const uint8_t* k8;                   // e4m3 codes and fp32 scales [L][Hkv] (KV8)
+  const uint8_t* v8;
+  const float* ksc;
+  const float* vsc;
   int64_t kv_tok, kv_head;
   const int32_t* idx;
   const int32_t* cnt;
@@ -74,6 +88,7 @@ struct FlashParams {
 };
 
 struct FlashBars {
+  uint64_t q_raw;  // KV8: Q landed (bf16), before its conversion
   uint64_t q_full;
   uint64_t full_k[FL_STAGES];
   uint64_t full_v[FL_STAGES];
@@ -92,6 +107,8 @@ constexpr uint32_t FL_BAR_OFF = FL_KV_OFF + FL_STAGES * 2 * TILE_BYTES;
 constexpr uint32_t FL_POS_OFF = FL_BAR_OFF + 256;
 constexpr uint32_t FL_SMEM_DENSE = FL_POS_OFF + 1024;  // + alignment slack
 constexpr uint32_t FL_SMEM_SPARSE = FL_POS_OFF + MAX_LIST * 4 + 1024;
+constexpr uint32_t FL_KSC_OFF = FL_POS_OFF + MAX_LIST * 4;  // KV8: [stage][128] column scales
+constexpr uint32_t FL_SMEM_KV8 = FL_KSC_OFF + FL_STAGES * 128 * 4 + 1024;
 
 // mbar_wait taken by every lane of a warp, with a warp-uniform result, for
 // roles that go on to issue warp-collective tcgen05.ld / tcgen05.st.
@@ -116,7 +133,7 @@ __device__ __forceinline__ bool wait_done(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
-template <int MODE>
+template <int MODE, bool KV8>
 __global__ void __launch_bounds__(FL_THREADS, 1)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const FlashParams p) {
@@ -124,6 +141,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
   uint8_t* smem = align1024(smem_raw);
   FlashBars* bars = reinterpret_cast<FlashBars*>(smem + FL_BAR_OFF);
   int32_t* pos_s = reinterpret_cast<int32_t*>(smem + FL_POS_OFF);
+  float* ksc_s = reinterpret_cast<float*>(smem + FL_KSC_OFF);
   const uint32_t q_base = smem_u32(smem + FL_Q_OFF);
   const uint32_t kv_base = smem_u32(smem + FL_KV_OFF);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -155,8 +173,9 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
   const bool has_b = (MODE == FLASH_DENSE) ? (nB > 0) : (2 * pair + 1 < p.mtiles);
 
   if (threadIdx.x == 0) {
-    const uint32_t kv_arrivals = (MODE == FLASH_DENSE) ? 1u : 64u;
-    mbar_init(&bars->q_full, 1);
+    const uint32_t kv_arrivals = (MODE == FLASH_DENSE && !KV8) ? 1u : 64u;
+    mbar_init(&bars->q_raw, 1);
+    mbar_init(&bars->q_full, KV8 ? 64u : 1u);
     for (int s = 0; s < FL_STAGES; ++s) {
       mbar_init(&bars->full_k[s], kv_arrivals);
       mbar_init(&bars->full_v[s], kv_arrivals);
@@ -185,19 +204,20 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     if (lane == 0 && !(p.flags & FLAG_SKIP_LOADS) && n > 0) {
       tma_prefetch_desc(&tmQ);
       const int nq = has_b ? 2 : 1;
-      mbar_arrive_expect_tx(&bars->q_full, static_cast<uint32_t>(nq) * TILE_BYTES);
+      uint64_t* qbar = KV8 ? &bars->q_raw : &bars->q_full;
+      mbar_arrive_expect_tx(qbar, static_cast<uint32_t>(nq) * TILE_BYTES);
       for (int x = 0; x < nq; ++x) {
         uint8_t* qd = smem + FL_Q_OFF + x * TILE_BYTES;
         if (MODE == FLASH_DENSE) {
-          tma_load_3d(qd, &tmQ, &bars->q_full, 0, h, (2 * pair + x) * 128);
-          tma_load_3d(qd + HALF_BYTES, &tmQ, &bars->q_full, 64, h, (2 * pair + x) * 128);
+          tma_load_3d(qd, &tmQ, qbar, 0, h, (2 * pair + x) * 128);
+          tma_load_3d(qd + HALF_BYTES, &tmQ, qbar, 64, h, (2 * pair + x) * 128);
         } else {
           const int t0 = 64 * b + (2 * pair + x) * p.rows_tok;
-          tma_load_3d(qd, &tmQ, &bars->q_full, 0, g * p.G, t0);
-          tma_load_3d(qd + HALF_BYTES, &tmQ, &bars->q_full, 64, g * p.G, t0);
+          tma_load_3d(qd, &tmQ, qbar, 0, g * p.G, t0);
+          tma_load_3d(qd + HALF_BYTES, &tmQ, qbar, 64, g * p.G, t0);
         }
       }
-      if (MODE == FLASH_DENSE) {
+      if (MODE == FLASH_DENSE && !KV8) {
         int last = -1;
         for (int j = 0; j < n; ++j) {
           const int s = j % FL_STAGES;
@@ -220,7 +240,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           wait_done(&bars->full_v[s], (j / FL_STAGES) & 1, p.limit_ns, 103);
         }
       }
-      wait_done(&bars->q_full, 0, p.limit_ns, 104);
+      wait_done(qbar, 0, p.limit_ns, 104);
     }
   } else if (warp == 1) {
     // ========================================================== MMA issue
@@ -232,8 +252,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t koff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + x * 128, sdesc_sw128(qb + koff, 16, 1024), sdesc_sw128(kb + koff, 16, 1024), IDESC_S,
-                  kk > 0 ? 1u : 0u);
+          umma_ss(tmem + x * 128, sdesc_sw128(qb + koff, 16, 1024), sdesc_sw128(kb + koff, 16, 1024),
+                  KV8 ? IDESC_S_F16 : IDESC_S, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bars->s_full[x]);
       };
@@ -242,7 +262,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bdesc = sdesc_sw128(vb + kk * 2048, HALF_BYTES, 1024);
-          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bdesc, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bdesc, KV8 ? IDESC_PV_F16 : IDESC_PV,
+                  (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars->o_done[x]);
       };
@@ -290,8 +311,77 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       wait_done(&bars->fin, 0, p.limit_ns, 116);
     }
   } else if (warp < 4) {
-    // ========================================================= K/V gather
-    if (MODE == FLASH_SPARSE && !(p.flags & FLAG_SKIP_LOADS)) {
+    // ============================================ KV8: convert Q, load K/V
+    if (KV8 && n > 0 && !(p.flags & FLAG_SKIP_LOADS)) {
+      const int pt = threadIdx.x - 64;  // 0..63
+      if (mbar_wait(&bars->q_raw, 0, p.limit_ns, abort_flag, 141)) {
+        const int nchunks = (has_b ? 2 : 1) * static_cast<int>(TILE_BYTES / 16);
+        for (int c = pt; c < nchunks; c += 64) {
+          const uint32_t a = q_base + c * 16;
+          st_shared_v4(a, bf16x8_to_f16x8(ld_shared_v4(a)));
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->q_full);
+        // K/V tiles: 8 threads per 128-byte code row, 16 codes -> two f16 chunks each
+        const int rsub = pt >> 3, c8 = pt & 7;
+        const uint8_t* kb8 = p.k8 + static_cast<int64_t>(g) * p.kv_head + c8 * 16;
+        const uint8_t* vb8 = p.v8 + static_cast<int64_t>(g) * p.kv_head + c8 * 16;
+        for (int j = 0; j < n; ++j) {
+          const int s = j % FL_STAGES;
+          if (j >= FL_STAGES &&
+              !mbar_wait(&bars->empty[s], ((j / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 142))
+            break;
+          const uint32_t kd = kv_base + s * 2 * TILE_BYTES;
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {  // 0: K, 1: V
+            const uint8_t* base8 = half ? vb8 : kb8;
+            const float* scale = half ? p.vsc : p.ksc;
+#pragma unroll 4
+            for (int it = 0; it < 16; ++it) {
+              const int r = rsub + 8 * it;
+              int pj;
+              bool valid;
+              if (MODE == FLASH_DENSE) {
+                pj = j * 128 + r;
+                valid = pj < p.L;
+              } else {
+                const int gi = j * 128 + r;
+                pj = pos_s[gi];
+                const bool listed = gi < cnt;
+                valid = listed && pj >= 0 && pj < e_b;
+                if (!half && listed && !valid) report(HS2_ERR_INDEX, 143);
+              }
+              uint4 raw = make_uint4(0, 0, 0, 0);
+              float sg = 0.f;
+              if (valid) {
+                raw = ld_nc_v4(base8 + static_cast<int64_t>(pj) * p.kv_tok);
+                sg = scale[static_cast<int64_t>(pj) * p.Hkv + g];
+              }
+              const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+              uint32_t f[8];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                f[2 * q] = e4m3x2_to_f16x2(w[q]);
+                f[2 * q + 1] = e4m3x2_to_f16x2(w[q] >> 16);
+              }
+              if (half) {
+                const uint32_t s2 = pack_f16x2(sg, sg);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) f[q] = hmul2_u32(f[q], s2);
+              } else if (c8 == 0) {
+                ksc_s[s * 128 + r] = sg * p.scale_log2;
+              }
+              const uint32_t dst = kd + half * TILE_BYTES;
+              st_shared_v4(dst + sw128_chunk_offset(r, 2 * c8, 128), make_uint4(f[0], f[1], f[2], f[3]));
+              st_shared_v4(dst + sw128_chunk_offset(r, 2 * c8 + 1, 128), make_uint4(f[4], f[5], f[6], f[7]));
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(half ? &bars->full_v[s] : &bars->full_k[s]);
+          }
+        }
+      }
+    } else if (MODE == FLASH_SPARSE && !KV8 && !(p.flags & FLAG_SKIP_LOADS)) {
+      // ========================================================= K/V gather
       const int pt = threadIdx.x - 64;  // 0..63
       const int row_sub = (pt >> 4) & 1, chunk = pt & 15, pw = pt >> 5;
       const __nv_bfloat16* kg = p.k + static_cast<int64_t>(g) * p.kv_head + chunk * 8;
@@ -358,7 +448,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       hh = g * p.G + r % p.G;
       i_min = 64 * b + mt * p.rows_tok;
     }
-    const float sc = p.scale_log2;
+    const float sc = KV8 ? 1.f : p.scale_log2;  // KV8 folds the scale into the columns
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nX; ++j) {
@@ -377,7 +467,22 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       reg_fence(sr[1]);
       reg_fence(sr[2]);
       reg_fence(sr[3]);
-      // ---- mask
+      if (KV8) {  // per-key scale (already times log2(e)/sqrt(d)) on every column
+        const uint64_t* ks2 = reinterpret_cast<const uint64_t*>(ksc_s + (j % FL_STAGES) * 128);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float a0, a1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])),
+                             ks2[c * 16 + e]),
+                      a0, a1);
+            sr[c][2 * e] = __float_as_uint(a0);
+            sr[c][2 * e + 1] = __float_as_uint(a1);
+          }
+        }
+      }
+      // ---- mask (after any scaling, so a masked column is exactly -inf)
       bool need_mask;
       if (MODE == FLASH_DENSE) {
         need_mask = (j == diag);
@@ -441,7 +546,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           sum2[e & 1] = f2_add(sum2[e & 1], p2);
           float e0, e1;
           f2_unpack(p2, e0, e1);
-          pk[e] = pack_bf16x2(e0, e1);
+          pk[e] = KV8 ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
         }
         tmem_st16(s_tm + c * 16, pk);
       }

@@ -62,7 +62,6 @@ int check_shape(const hs2_shape* s) {
   if (s->q_head_stride < HD || s->kv_head_stride < HD) return HS2_ERR_UNSUPPORTED;
   if (s->q_tok_stride < static_cast<int64_t>(s->Hq) * s->q_head_stride) return HS2_ERR_UNSUPPORTED;
   if (s->kv_tok_stride < static_cast<int64_t>(s->Hkv) * s->kv_head_stride) return HS2_ERR_UNSUPPORTED;
-  if (s->kv_dtype == HS2_KV_E4M3) return HS2_ERR_UNSUPPORTED;  // FP8 cache: not built yet
   return HS2_OK;
 }
 
@@ -117,14 +116,26 @@ int set_smem(K kernel, uint32_t bytes) {
 
 // ------------------------------------------------------------- launches --
 
-int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void* v, void* o, float* lse,
-                    cudaStream_t st) {
+int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void* v, const float* ks,
+                    const float* vs, void* o, float* lse, cudaStream_t st) {
+  const bool kv8 = s->kv_dtype == HS2_KV_E4M3;
   CUtensorMap mq, mk, mv;
   int rc;
   if ((rc = make_map(&mq, q, s->L, s->Hq, s->q_tok_stride, s->q_head_stride, 1, 128))) return rc;
-  if ((rc = make_map(&mk, k, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
-  if ((rc = make_map(&mv, v, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+  if (!kv8) {
+    if ((rc = make_map(&mk, k, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+    if ((rc = make_map(&mv, v, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+  } else {
+    mk = mq;
+    mv = mq;
+  }
   FlashParams p{};
+  p.k8 = static_cast<const uint8_t*>(k);
+  p.v8 = static_cast<const uint8_t*>(v);
+  p.ksc = ks;
+  p.vsc = vs;
+  p.kv_tok = s->kv_tok_stride;
+  p.kv_head = s->kv_head_stride;
   p.L = s->L;
   p.Hq = s->Hq;
   p.Hkv = s->Hkv;
@@ -138,15 +149,21 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
   p.lse = lse;
   p.limit_ns = g_wait_limit_ns;
   p.flags = g_flags;
-  static int attr = set_smem(flash_fwd_kernel<FLASH_DENSE>, FL_SMEM_DENSE);
-  if (attr) return attr;
   const unsigned grid = static_cast<unsigned>(p.npairs * s->Hq);
-  flash_fwd_kernel<FLASH_DENSE><<<grid, FL_THREADS, FL_SMEM_DENSE, st>>>(mq, mk, mv, p);
+  if (kv8) {
+    static int attr8 = set_smem(flash_fwd_kernel<FLASH_DENSE, true>, FL_SMEM_KV8);
+    if (attr8) return attr8;
+    flash_fwd_kernel<FLASH_DENSE, true><<<grid, FL_THREADS, FL_SMEM_KV8, st>>>(mq, mk, mv, p);
+  } else {
+    static int attr = set_smem(flash_fwd_kernel<FLASH_DENSE, false>, FL_SMEM_DENSE);
+    if (attr) return attr;
+    flash_fwd_kernel<FLASH_DENSE, false><<<grid, FL_THREADS, FL_SMEM_DENSE, st>>>(mq, mk, mv, p);
+  }
   return launched();
 }
 
-int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* v, const int32_t* idx,
-                  const int32_t* cnt, void* o, cudaStream_t st) {
+int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* v, const float* ks,
+                  const float* vs, const int32_t* idx, const int32_t* cnt, void* o, cudaStream_t st) {
   const int G = s->Hq / s->Hkv;
   const int rows_tok = 128 / G;
   CUtensorMap mq;
@@ -165,6 +182,10 @@ int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* 
   p.scale_log2 = scale_log2(s->d);
   p.k = static_cast<const __nv_bfloat16*>(k);
   p.v = static_cast<const __nv_bfloat16*>(v);
+  p.k8 = static_cast<const uint8_t*>(k);
+  p.v8 = static_cast<const uint8_t*>(v);
+  p.ksc = ks;
+  p.vsc = vs;
   p.kv_tok = s->kv_tok_stride;
   p.kv_head = s->kv_head_stride;
   p.idx = idx;
@@ -174,34 +195,49 @@ int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* 
   p.o_head = s->q_head_stride;
   p.limit_ns = g_wait_limit_ns;
   p.flags = g_flags;
-  static int attr = set_smem(flash_fwd_kernel<FLASH_SPARSE>, FL_SMEM_SPARSE);
-  if (attr) return attr;
   const unsigned grid = static_cast<unsigned>(p.nb * s->Hkv * p.mpairs);
-  flash_fwd_kernel<FLASH_SPARSE><<<grid, FL_THREADS, FL_SMEM_SPARSE, st>>>(mq, mq, mq, p);
+  if (s->kv_dtype == HS2_KV_E4M3) {
+    static int attr8 = set_smem(flash_fwd_kernel<FLASH_SPARSE, true>, FL_SMEM_KV8);
+    if (attr8) return attr8;
+    flash_fwd_kernel<FLASH_SPARSE, true><<<grid, FL_THREADS, FL_SMEM_KV8, st>>>(mq, mq, mq, p);
+  } else {
+    static int attr = set_smem(flash_fwd_kernel<FLASH_SPARSE, false>, FL_SMEM_SPARSE);
+    if (attr) return attr;
+    flash_fwd_kernel<FLASH_SPARSE, false><<<grid, FL_THREADS, FL_SMEM_SPARSE, st>>>(mq, mq, mq, p);
+  }
   return launched();
 }
 
 int n_cand(const hs2_shape* s, int b) { return std::max(0, std::min(s->L, 64 * (b + 1)) - s->recent); }
 
-template <int G>
+template <int G, bool KV8>
 int launch_importance_g(const CUtensorMap& mq, const CUtensorMap& mk, const ImpParams& p, dim3 grid,
                         cudaStream_t st) {
-  static int attr = set_smem(importance_kernel<G>, imp_smem_bytes(G));
+  static int attr = set_smem(importance_kernel<G, KV8>, imp_smem_bytes(G));
   if (attr) return attr;
-  importance_kernel<G><<<grid, IMP_THREADS, imp_smem_bytes(G), st>>>(mq, mk, p);
+  importance_kernel<G, KV8><<<grid, IMP_THREADS, imp_smem_bytes(G), st>>>(mq, mk, p);
   return launched();
 }
 
-int launch_importance(const hs2_shape* s, const void* q, const void* k, const float* lse, int b0, int b1,
-                      float* imp, int64_t row_stride, int skip_le, cudaStream_t st) {
+int launch_importance(const hs2_shape* s, const void* q, const void* k, const float* ks, const float* lse, int b0,
+                      int b1, float* imp, int64_t row_stride, int skip_le, cudaStream_t st) {
+  const bool kv8 = s->kv_dtype == HS2_KV_E4M3;
   const int G = s->Hq / s->Hkv;
   const int longest = n_cand(s, b1 - 1);
   if (longest <= 0 || longest <= skip_le) return HS2_OK;
   CUtensorMap mq, mk;
   int rc;
   if ((rc = make_map(&mq, q, s->L, s->Hq, s->q_tok_stride, s->q_head_stride, G, 64))) return rc;
-  if ((rc = make_map(&mk, k, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+  if (!kv8) {
+    if ((rc = make_map(&mk, k, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+  } else {
+    mk = mq;
+  }
   ImpParams p{};
+  p.k8 = static_cast<const uint8_t*>(k);
+  p.ksc = ks;
+  p.kv_tok = s->kv_tok_stride;
+  p.kv_head = s->kv_head_stride;
   p.L = s->L;
   p.Hq = s->Hq;
   p.Hkv = s->Hkv;
@@ -217,10 +253,13 @@ int launch_importance(const hs2_shape* s, const void* q, const void* k, const fl
   p.limit_ns = g_wait_limit_ns;
   p.flags = g_flags;
   const dim3 grid(static_cast<unsigned>((longest + IMP_CK - 1) / IMP_CK), static_cast<unsigned>(s->Hkv * (b1 - b0)));
-  switch (G) {
-    case 2: return launch_importance_g<2>(mq, mk, p, grid, st);
-    case 4: return launch_importance_g<4>(mq, mk, p, grid, st);
-    case 8: return launch_importance_g<8>(mq, mk, p, grid, st);
+  switch (G * 2 + (kv8 ? 1 : 0)) {
+    case 4: return launch_importance_g<2, false>(mq, mk, p, grid, st);
+    case 5: return launch_importance_g<2, true>(mq, mk, p, grid, st);
+    case 8: return launch_importance_g<4, false>(mq, mk, p, grid, st);
+    case 9: return launch_importance_g<4, true>(mq, mk, p, grid, st);
+    case 16: return launch_importance_g<8, false>(mq, mk, p, grid, st);
+    case 17: return launch_importance_g<8, true>(mq, mk, p, grid, st);
     default: return HS2_ERR_UNSUPPORTED;
   }
 }
@@ -342,7 +381,7 @@ int hs2_attn_fwd(const hs2_shape* shape, const void* q, const void* k, const voi
   if ((rc = check_kv(shape, k, v, k_scale, v_scale))) return rc;
   if (!q || !o || !lse) return HS2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || !aligned16(lse)) return HS2_ERR_UNSUPPORTED;
-  return launch_attn_fwd(shape, q, k, v, o, lse, static_cast<cudaStream_t>(stream));
+  return launch_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, static_cast<cudaStream_t>(stream));
 }
 
 int hs2_importance(const hs2_shape* shape, const void* q, const void* k, const float* k_scale, const float* lse,
@@ -355,7 +394,8 @@ int hs2_importance(const hs2_shape* shape, const void* q, const void* k, const f
   if (b0 < 0 || b1 > nb || b0 >= b1) return HS2_ERR_INVALID_ARG;
   if (row_stride % 4 || row_stride < n_cand(shape, b1 - 1)) return HS2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(imp)) return HS2_ERR_UNSUPPORTED;
-  return launch_importance(shape, q, k, lse, b0, b1, imp, row_stride, -1, static_cast<cudaStream_t>(stream));
+  return launch_importance(shape, q, k, k_scale, lse, b0, b1, imp, row_stride, -1,
+                           static_cast<cudaStream_t>(stream));
 }
 
 int hs2_topk_select(const hs2_shape* shape, const float* imp, int64_t row_stride, int32_t b0, int32_t b1,
@@ -386,7 +426,7 @@ int hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, c
   const size_t ws = *workspace_bytes;
   if (ws < min_workspace(shape)) return HS2_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((rc = launch_attn_fwd(shape, q, k, v, o, lse, st))) return rc;
+  if ((rc = launch_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, st))) return rc;
 
   // Strips of query blocks.  Blocks whose candidates all fit in the top-k
   // need no importance; the rest are grouped so that a strip's rows
@@ -402,7 +442,7 @@ int hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, c
     } else {
       while (b1 < nb && static_cast<size_t>(shape->Hkv) * (b1 + 1 - b) * strip_stride(shape, b1) * 4u <= ws) ++b1;
       const int64_t stride = strip_stride(shape, b1 - 1);
-      if ((rc = launch_importance(shape, q, k, lse, b, b1, imp, stride, shape->topk, st))) return rc;
+      if ((rc = launch_importance(shape, q, k, k_scale, lse, b, b1, imp, stride, shape->topk, st))) return rc;
       if ((rc = launch_select(shape, imp, stride, b, b1, idx, cnt, st))) return rc;
     }
     b = b1;
@@ -429,7 +469,7 @@ int hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const 
   if ((rc = check_kv(shape, k, v, k_scale, v_scale))) return rc;
   if (!q || !o || !idx || !cnt) return HS2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || !aligned16(idx)) return HS2_ERR_UNSUPPORTED;
-  return launch_sparse(shape, q, k, v, idx, cnt, o, static_cast<cudaStream_t>(stream));
+  return launch_sparse(shape, q, k, v, k_scale, v_scale, idx, cnt, o, static_cast<cudaStream_t>(stream));
 }
 
 int hs2_sync(void* stream) {

@@ -24,6 +24,9 @@
 // memory, which adds them in a fixed order (the result is deterministic, so
 // hs2_importance reproduces exactly what the selection saw).  Arguments and
 // sums use packed f32x2 FMA/ADD; the exponentials run on the MUFU unit.
+// FP8 e4m3 cache (KV8): warps 2-3 convert the Q block to f16 in place and
+// convert each K tile exactly from e4m3 to f16 (MMAs run kind::f16); each
+// key's fp32 scale multiplies its row of scores in the epilogue.
 // Work item = (KV head, block, chunk of IMP_CK keys); the grid is
 // (chunks of the longest row of the strip) x (Hkv * blocks).
 #pragma once
@@ -38,6 +41,9 @@ constexpr int IMP_STAGES = 2;  // K tile ring (deeper rings measured no faster)
 
 struct ImpParams {
   int L, Hq, Hkv, G, recent, b0, nbs;
+  const uint8_t* k8;  // e4m3 K codes and fp32 scales [L][Hkv] (KV8)
+  const float* ksc;
+  int64_t kv_tok, kv_head;
   int skip_le;       // rows with |C_b| <= skip_le are not computed (-1: compute all)
   float scale_log2;  // log2(e) / sqrt(d)
   const float* lse;  // [Hq][L]
@@ -48,6 +54,7 @@ struct ImpParams {
 };
 
 struct ImpBars {
+  uint64_t q_raw;  // KV8: Q block landed (bf16), before its conversion to f16
   uint64_t q_full;
   uint64_t k_full[IMP_STAGES];
   uint64_t k_empty[IMP_STAGES];
@@ -71,7 +78,7 @@ __host__ __device__ constexpr uint32_t imp_smem_bytes(int G) {
   return imp_part_off(G) + (IMP_GROUPS - 1) * 2u * 128u * 4u + 1024u;
 }
 
-template <int G>
+template <int G, bool KV8>
 __global__ void __launch_bounds__(IMP_THREADS, 1)
     importance_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const ImpParams p) {
@@ -79,7 +86,7 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
   constexpr int NSUB = (NQ < 256) ? NQ : 256;   // MMA N per sub-tile
   constexpr int SUBS = NQ / NSUB;
   constexpr uint32_t QHALF = static_cast<uint32_t>(NQ) * 128u;
-  constexpr uint32_t IDESC = idesc_bf16_f32(128, NSUB, 0, 0);
+  constexpr uint32_t IDESC = KV8 ? idesc_f16_f32(128, NSUB, 0, 0) : idesc_bf16_f32(128, NSUB, 0, 0);
   constexpr uint32_t TMEM_COLS = (2 * NSUB <= 256) ? 256u : 512u;
 
   const int y = blockIdx.y;
@@ -102,9 +109,10 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
   volatile int* abort_flag = &bars->abort;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_raw, 1);
+    mbar_init(&bars->q_full, KV8 ? 64u : 1u);
     for (int s = 0; s < IMP_STAGES; ++s) {
-      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_full[s], KV8 ? 64u : 1u);
       mbar_init(&bars->k_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -135,11 +143,12 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
     if (lane == 0 && !(p.flags & FLAG_SKIP_LOADS)) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
-      mbar_arrive_expect_tx(&bars->q_full, 2 * QHALF);
-      tma_load_3d(smem, &tmQ, &bars->q_full, 0, g * G, 64 * b);
-      tma_load_3d(smem + QHALF, &tmQ, &bars->q_full, 64, g * G, 64 * b);
+      uint64_t* qbar = KV8 ? &bars->q_raw : &bars->q_full;
+      mbar_arrive_expect_tx(qbar, 2 * QHALF);
+      tma_load_3d(smem, &tmQ, qbar, 0, g * G, 64 * b);
+      tma_load_3d(smem + QHALF, &tmQ, qbar, 64, g * G, 64 * b);
       int last = -1;
-      for (int t = 0; t < ntiles; ++t) {
+      for (int t = 0; t < (KV8 ? 0 : ntiles); ++t) {
         const int s = t % IMP_STAGES;
         if (t >= IMP_STAGES &&
             !mbar_wait(&bars->k_empty[s], ((t / IMP_STAGES) - 1) & 1, p.limit_ns, abort_flag, 201))
@@ -152,7 +161,7 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
       }
       for (int t = max(0, last - IMP_STAGES + 1); t <= last; ++t)
         wait_done(&bars->k_full[t % IMP_STAGES], (t / IMP_STAGES) & 1, p.limit_ns, 202);
-      wait_done(&bars->q_full, 0, p.limit_ns, 203);
+      wait_done(qbar, 0, p.limit_ns, 203);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -189,6 +198,45 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
       umma_commit(&bars->fin);
       wait_done(&bars->fin, 0, p.limit_ns, 214);
     }
+  } else if (warp < 4) {
+    // KV8: convert the Q block to f16 in place, then load, convert (exactly,
+    // e4m3 -> f16) and store every K tile; 8 threads per 128-byte code row.
+    if (KV8 && !(p.flags & FLAG_SKIP_LOADS)) {
+      const int pt = threadIdx.x - 64;
+      if (mbar_wait(&bars->q_raw, 0, p.limit_ns, abort_flag, 241)) {
+        for (int c = pt; c < static_cast<int>(2 * QHALF / 16); c += 64) {
+          const uint32_t a = q_base + c * 16;
+          st_shared_v4(a, bf16x8_to_f16x8(ld_shared_v4(a)));
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->q_full);
+        const int rsub = pt >> 3, c8 = pt & 7;
+        const uint8_t* kb8 = p.k8 + static_cast<int64_t>(g) * p.kv_head + c8 * 16;
+        for (int t = 0; t < ntiles; ++t) {
+          const int s = t % IMP_STAGES;
+          if (t >= IMP_STAGES &&
+              !mbar_wait(&bars->k_empty[s], ((t / IMP_STAGES) - 1) & 1, p.limit_ns, abort_flag, 242))
+            break;
+          const uint32_t kd = k_base + s * TILE_BYTES;
+#pragma unroll 4
+          for (int it = 0; it < 16; ++it) {
+            const int r = rsub + 8 * it;
+            const uint4 raw = ld_nc_v4(kb8 + static_cast<int64_t>(j0 + t * 128 + r) * p.kv_tok);  // < L
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+            uint32_t f[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              f[2 * q] = e4m3x2_to_f16x2(w[q]);
+              f[2 * q + 1] = e4m3x2_to_f16x2(w[q] >> 16);
+            }
+            st_shared_v4(kd + sw128_chunk_offset(r, 2 * c8, 128), make_uint4(f[0], f[1], f[2], f[3]));
+            st_shared_v4(kd + sw128_chunk_offset(r, 2 * c8 + 1, 128), make_uint4(f[4], f[5], f[6], f[7]));
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&bars->k_full[s]);
+        }
+      }
+    }
   } else if (warp >= 4) {
     const int grp = (warp - 4) >> 2;              // epilogue group 0..IMP_GROUPS-1
     const int r = threadIdx.x - 128 - 128 * grp;  // key row of the tile
@@ -201,6 +249,12 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) {
       uint64_t acc2[2] = {0ull, 0ull};
+      uint64_t c2t = c2p;
+      if (KV8) {  // this key's scale multiplies its whole row of scores
+        const int jk = min(j0 + t * 128 + r, p.L - 1);
+        const float cs = p.scale_log2 * p.ksc[static_cast<int64_t>(jk) * p.Hkv + g];
+        c2t = f2_pack(cs, cs);
+      }
       for (int sub = 0; sub < SUBS; ++sub, ++u) {
         const int buf = u & 1;
         if (!warp_wait(&bars->acc_full[buf], (u >> 1) & 1, p.limit_ns, abort_flag, 221)) {
@@ -224,9 +278,9 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
           for (int e4 = 0; e4 < 8; ++e4) {
             const float4 nl = nl4[c * 8 + e4];  // broadcast read
             const uint64_t a01 = f2_fma(f2_pack(__uint_as_float(sr[c][4 * e4]), __uint_as_float(sr[c][4 * e4 + 1])),
-                                        c2p, f2_pack(nl.x, nl.y));
+                                        c2t, f2_pack(nl.x, nl.y));
             const uint64_t a23 = f2_fma(
-                f2_pack(__uint_as_float(sr[c][4 * e4 + 2]), __uint_as_float(sr[c][4 * e4 + 3])), c2p,
+                f2_pack(__uint_as_float(sr[c][4 * e4 + 2]), __uint_as_float(sr[c][4 * e4 + 3])), c2t,
                 f2_pack(nl.z, nl.w));
             acc2[0] = f2_add(acc2[0], ex2_x2(a01));
             acc2[1] = f2_add(acc2[1], ex2_x2(a23));
