@@ -68,6 +68,29 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# ------------------------------------------------------------ multi-rank --
+
+def rank_workload(wl, rank: int, world: int):
+    """Each rank prefills its own independent sequence (a batch of `world`
+    sequences, one per GPU): same shapes, its own seed."""
+    return wl.scaled(seed=wl.seed + 101 * rank) if world > 1 else wl
+
+
+def reduce_max(value: float, dist, device=None) -> float:
+    """Max of a per-rank timing over all ranks (identity without a group)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], device=device if device is not None else "cpu", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(L: int, world: int, ms: float) -> float:
+    """Whole-job tokens/s: every rank processed L tokens in at most `ms`."""
+    return world * L / (ms / 1e3)
+
+
 # ---------------------------------------------------------------- clocks --
 
 class ClockSampler:
@@ -221,7 +244,7 @@ def run_cuda(args, wl, rank, world, dist):
     build.build()
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    my = wl.scaled(seed=wl.seed + 101 * rank) if world > 1 else wl
+    my = rank_workload(wl, rank, world)
     x = inputs.make_inputs(my, device=dev, with_needles=bool(my.needles))
     q0, k, v = x["q_layers"][0], x["k"], x["v"]
     shape = hs2.make_shape(q0, k, wl.topk, wl.recent)
@@ -258,11 +281,7 @@ def run_cuda(args, wl, rank, world, dist):
     launches = hs2.hs2_launch_count() - n0
     hs2.hs2_sync(stream)
     per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = ev[0].elapsed_time(ev[-1])
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(ev[0].elapsed_time(ev[-1]), dist, dev)
     ms = total_ms / args.steps
 
     # ---- per-stage device times (same stream, CUDA events), full kernel (1)
@@ -314,13 +333,9 @@ def run_cuda(args, wl, rank, world, dist):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b) / n_e2e
-        if dist is not None:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = reduce_max(a.elapsed_time(b) / n_e2e, dist, dev)
         hs2.hs2_sync(stream)
-        e2e = {"value": world * wl.L / (e_ms / 1e3), "unit": "tok/s",
+        e2e = {"value": job_throughput(wl.L, world, e_ms), "unit": "tok/s",
                "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in h_in)),
                "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in h_out)), "ms_per_step": e_ms}
         del h_in, h_out, d_in
@@ -330,7 +345,7 @@ def run_cuda(args, wl, rank, world, dist):
     fa_tflops = work["fa_flop"] / (fa_ms / 1e3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     res = {
-        "metric": METRIC, "value": world * wl.L / (ms / 1e3), "unit": "tok/s", "n_gpus": world,
+        "metric": METRIC, "value": job_throughput(wl.L, world, ms), "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "p50_ms": float(np.percentile(per, 50)), "p99_ms": float(np.percentile(per, 99)),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
