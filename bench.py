@@ -59,6 +59,37 @@ def algorithmic_work(wl) -> dict:
             "gather_bytes": gather, "sparse_qo_bytes": qo}
 
 
+FA_SOURCES = ("token_level_sparse_causal_b200/csrc/flash.cuh", "token_level_sparse_causal_b200/csrc/common.cuh")
+FA_TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "flash_fwd_dense_dram_L131072.md")
+
+
+def kernel_source_hash(paths=FA_SOURCES) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(profile=FA_TRAFFIC_PROFILE):
+    """DRAM bytes per launch of kernel (1) from the committed ncu summary, or
+    None when the kernel sources changed since those counters were taken."""
+    if not os.path.exists(profile):
+        return None
+    fields = {}
+    for line in open(profile):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            fields[k.strip()] = v.strip()
+    if fields.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -356,7 +387,7 @@ def run_cuda(args, wl, rank, world, dist):
                    "l2": "inputs larger than L2 (Q alone is %.1f GB); no flush" % (q0.numel() * 2 / 1e9)},
         "roofline": {"kernel": "fa_fwd (kernel 1, dense causal attention + LSE)", "bound": "tensor",
                      "achieved": fa_tflops, "peak": peak, "unit": "TFLOP/s", "frac": fa_tflops / peak,
-                     "traffic": None,
+                     "traffic": recorded_traffic(), "traffic_unit": "bytes per launch (dram read + write, ncu)",
                      "peak_note": f"{peaks['source']} sustained bf16 (the kernel runs ~{fa_ms:.0f} ms per launch)"},
         "stages_ms": {"fa_fwd": fa_ms, "importance+select": fs_ms - fa_ms, "sparse_attn_per_layer": sp_ms,
                       "full_attn_select": fs_ms},

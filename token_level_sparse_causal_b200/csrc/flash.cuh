@@ -150,9 +150,13 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
   // ---- work item: query tiles A and B (B may be absent), key tiles nA / nB
   int h = 0, g = 0, b = 0, pair = 0, cnt = 0, e_b = 0, nA = 0, nB = 0;
   if (MODE == FLASH_DENSE) {
-    pair = p.npairs - 1 - static_cast<int>(blockIdx.x) / p.Hq;  // longest rows first
-    h = static_cast<int>(blockIdx.x) % p.Hq;
-    g = h / p.G;
+    // KV-group-major order, longest tile pairs first within a group: the
+    // CTAs resident at any time share one group's K/V, which then stays in L2.
+    const int per_g = p.npairs * p.G;
+    g = static_cast<int>(blockIdx.x) / per_g;
+    const int rem = static_cast<int>(blockIdx.x) % per_g;
+    pair = p.npairs - 1 - rem / p.G;
+    h = g * p.G + rem % p.G;
     nA = 2 * pair + 1;
     nB = (2 * pair + 1 < p.nqt) ? 2 * pair + 2 : 0;
   } else {
