@@ -76,6 +76,44 @@ def dequantize(codes_u8: np.ndarray, scale: np.ndarray) -> np.ndarray:
     return decode_e4m3(codes_u8) * np.asarray(scale, dtype=np.float64)[..., None]
 
 
+E4M3_MAX = 448.0
+
+
+def _e4m3_grid() -> np.ndarray:
+    """All non-negative finite e4m3fn values, ascending (code order)."""
+    return decode_e4m3(np.arange(0x7F, dtype=np.uint8))   # 0x00..0x7E; 0x7F is NaN
+
+
+def encode_e4m3(y) -> np.ndarray:
+    """Round values to OCP e4m3fn codes: nearest representable value, ties to
+    the even code (mantissa LSB 0), magnitudes beyond 448 saturate to 448
+    (reading R10); the sign bit follows the input's sign, zero included.
+    Works on float32 inputs exactly, by search over the grid."""
+    y = np.asarray(y, dtype=np.float64)
+    grid = _e4m3_grid()
+    mag = np.minimum(np.abs(y), E4M3_MAX)
+    hi = np.clip(np.searchsorted(grid, mag, side="left"), 1, grid.size - 1)
+    lo = hi - 1
+    d_lo, d_hi = mag - grid[lo], grid[hi] - mag
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(mag <= 0.0, 0, np.where(mag >= grid[-1], grid.size - 1, np.where(take_hi, hi, lo)))
+    sign = np.where(np.signbit(y), 0x80, 0)   # a negative value keeps its sign, even at zero
+    return (code | sign).astype(np.uint8)
+
+
+def quantize_kv(x_rows):
+    """FP8 KV write (HS2 cost paragraph: FP8 KV cache; reading R10): for each
+    row of 128 values (one token, one KV head), scale = amax / 448 computed in
+    float32 (1 when the row is all zero), codes = e4m3(x / scale) with the
+    division in float32.  x_rows [..., d] holds values exactly representable in
+    float32.  Returns (codes uint8 [..., d], scale float32 [...])."""
+    x = np.asarray(x_rows, dtype=np.float32)
+    amax = np.abs(x).max(axis=-1)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    y = (x / scale[..., None]).astype(np.float32)
+    return encode_e4m3(y), scale
+
+
 # ------------------------------------------------------- index arithmetic --
 
 

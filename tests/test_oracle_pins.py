@@ -392,3 +392,43 @@ def test_planted_mistakes_are_caught():
     assert check_select_brute(_sel_rev) > 0
     assert check_select_brute(_select_no_recent) > 0
     assert check_sparse_vs_masked_sdpa(_sparse_unmasked) > 1e-3
+
+
+# ------------------------------------------------------------ FP8 KV write --
+
+def test_encode_e4m3_matches_torch_round_to_nearest_even():
+    rng = np.random.default_rng(7)
+    y = np.concatenate([rng.standard_normal(200_000) * 100, rng.uniform(-448, 448, 200_000),
+                        rng.uniform(-2.0 ** -6, 2.0 ** -6, 50_000)]).astype(np.float32)
+    grid = orc.decode_e4m3(np.arange(0x7F, dtype=np.uint8))
+    mids = ((grid[1:] + grid[:-1]) / 2).astype(np.float32)        # exact ties (representable in fp32)
+    y = np.concatenate([y, mids, -mids, [0.0, -0.0, 2.0 ** -11, -(2.0 ** -11)]]).astype(np.float32)
+    y = np.clip(y, -448, 448)
+    ref = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = orc.encode_e4m3(y)
+    assert np.array_equal(got, ref)
+
+
+def test_encode_decode_roundtrip_and_saturation():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    vals = orc.decode_e4m3(codes)
+    back = orc.encode_e4m3(vals)
+    assert np.array_equal(orc.decode_e4m3(back), vals)
+    assert orc.decode_e4m3(orc.encode_e4m3(np.array([1e6, -1e6, 449.0])))[0] == 448.0
+    assert orc.decode_e4m3(orc.encode_e4m3(np.array([-1e6])))[0] == -448.0
+
+
+def test_quantize_kv_row_definition():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((64, 3, 128)).astype(np.float32)
+    x[5, 1] = 0.0
+    codes, scale = orc.quantize_kv(x)
+    assert scale.dtype == np.float32 and scale[5, 1] == 1.0
+    amax = np.abs(x).max(axis=-1)
+    nz = amax > 0
+    assert np.array_equal(scale[nz], (amax / np.float32(448)).astype(np.float32)[nz])
+    deq = orc.dequantize(codes, scale)
+    # every element within half an e4m3 step of its value; the row max lands on 448 * scale
+    assert np.all(np.abs(deq - x) <= np.abs(x) * 2.0 ** -4 + scale[..., None] * 2.0 ** -9 + 1e-12)
+    top = np.abs(x).argmax(axis=-1)
+    assert np.all(np.abs(np.take_along_axis(orc.decode_e4m3(codes), top[..., None], -1)[..., 0][nz]) == 448.0)
