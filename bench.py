@@ -328,6 +328,16 @@ def run_cuda(args, wl, rank, world, dist):
         return a.elapsed_time(b) / n
 
     n_stage = max(2, min(args.steps, 5))
+    # FP8 KV write (the step producing an e4m3 cache) on this workload's K
+    fp8 = None
+    if k.dtype == torch.bfloat16:
+        codes = torch.empty(k.shape, dtype=torch.uint8, device=dev)
+        kscale = torch.empty(k.shape[:2], dtype=torch.float32, device=dev)
+        qk_ms = timed(lambda: hs2.hs2_quantize_kv(k, codes, kscale, stream), n_stage)
+        moved = k.numel() * 2 + codes.numel() + kscale.numel() * 4
+        fp8 = {"ms": qk_ms, "gbs": moved / (qk_ms / 1e3) / 1e9, "frac_of_hbm": moved / (qk_ms / 1e3) / 1e9 /
+               measured_peaks()["hbm_gbs"], "bytes": moved}
+        del codes, kscale
     fa_ms = timed(lambda: hs2.hs2_attn_fwd(shape, q0, k, v, None, None, out["o"], out["lse"], stream), n_stage)
     sp_ms = timed(lambda: hs2.hs2_sparse_attn(shape, x["q_layers"][1], k, v, None, None, out["idx"], out["cnt"],
                                               o_sp[0], stream), n_stage) if o_sp else 0.0
@@ -400,6 +410,7 @@ def run_cuda(args, wl, rank, world, dist):
                                        (peaks["bf16_tflops_sustained"] * 1e12) +
                                        2 * work["select_bytes"] / (peaks["hbm_gbs"] * 1e9)),
         },
+        "next_rows": {"fp8_kv_write_K": fp8},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "e2e": e2e,

@@ -138,6 +138,20 @@ int hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const 
                     void* o, void* stream);
 
 /*
+ * FP8 KV write: quantise a bf16 K or V cache to OCP e4m3fn codes with one fp32
+ * scale per (token, KV head), the format hs2_shape.kv_dtype = HS2_KV_E4M3 reads
+ * (HySparse2 architecture summary, cost paragraph: FP8 KV cache).  For each row
+ * of d = 128 values: scale = amax / 448 in fp32 (1 for an all-zero row),
+ * code = e4m3(x / scale) with fp32 division and saturating round-to-nearest-
+ * even.  src: bf16 [L][Hkv][128], element strides (multiples of 8, base
+ * 16-byte aligned); dst: uint8 [L][Hkv][128], byte strides (multiples of 8,
+ * base 8-byte aligned); scale: fp32 [L][Hkv] contiguous.  Device pointers;
+ * asynchronous on `stream`.
+ */
+int hs2_quantize_kv(int32_t L, int32_t Hkv, const void* src, int64_t src_tok_stride, int64_t src_head_stride,
+                    void* dst, int64_t dst_tok_stride, int64_t dst_head_stride, float* scale, void* stream);
+
+/*
  * Blocks until `stream` is idle, then returns the first error recorded on the
  * device since the previous hs2_sync (and clears it), or HS2_ERR_CUDA if the
  * stream reported an error, else HS2_OK.

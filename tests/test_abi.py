@@ -141,3 +141,14 @@ def test_fp8_needs_scales(lib):
 def test_debug_set_validates(lib):
     assert lib.hs2_debug_set(0, 0) == hs2.HS2_ERR_INVALID_ARG
     assert lib.hs2_debug_set(2_000_000_000, 0) == hs2.HS2_OK
+
+
+def test_quantize_kv_argument_checks(lib):
+    st = ctypes.c_void_p(0)
+    assert lib.hs2_quantize_kv(0, 2, P, 256, 128, P, 256, 128, P, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_quantize_kv(16, 2, None, 256, 128, P, 256, 128, P, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_quantize_kv(16, 2, P, 256, 64, P, 256, 128, P, st) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_quantize_kv(16, 2, P, 200, 128, P, 256, 128, P, st) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_quantize_kv(16, 2, ctypes.c_void_p(0x10008), 256, 128, P, 256, 128, P, st) == \
+        hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_quantize_kv(16, 2, P, 256, 128, P, 260, 128, P, st) == hs2.HS2_ERR_UNSUPPORTED

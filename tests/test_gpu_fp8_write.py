@@ -1,0 +1,66 @@
+"""FP8 KV write (hs2_quantize_kv) against the oracle's quantiser: codes and
+scales bit-exact (both sides divide in fp32 and round to nearest even)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import hs2_oracle as orc
+from token_level_sparse_causal_b200 import build, hs2, inputs
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build.build()
+    hs2.hs2_debug_set(500_000_000, 0)
+
+
+def _check(src_bf16, dst, scale):
+    codes, sc = orc.quantize_kv(orc.decode_bf16(inputs.as_u16(src_bf16)))
+    assert np.array_equal(scale.cpu().numpy(), sc)
+    assert np.array_equal(dst.cpu().numpy(), codes)
+
+
+def test_random_rows_with_zeros_and_extremes():
+    g = torch.Generator().manual_seed(11)
+    x = (torch.randn((777, 3, 128), generator=g) * torch.logspace(-3, 3, 777)[:, None, None]).to(torch.bfloat16)
+    x[5] = 0
+    x[6, 1, :] = -0.0
+    x[7, 2, 3] = 3.0e38
+    x[8, 0, ::2] = -1e-30
+    xd = x.to(DEV)
+    dst = torch.full((777, 3, 128), 0xAA, dtype=torch.uint8, device=DEV)
+    scale = torch.empty((777, 3), device=DEV)
+    hs2.hs2_quantize_kv(xd, dst, scale)
+    hs2.hs2_sync()
+    _check(x, dst, scale)
+
+
+def test_padded_strides_leave_padding_untouched():
+    g = torch.Generator().manual_seed(12)
+    big = torch.randn((301, 5, 136), generator=g).to(torch.bfloat16).to(DEV)
+    src = big[:301, 1:4, :128]
+    out = torch.full((301, 4, 136), 0x5A, dtype=torch.uint8, device=DEV)
+    dst = out[:, :3, :128]
+    scale = torch.empty((301, 3), device=DEV)
+    hs2.hs2_quantize_kv(src, dst, scale)
+    hs2.hs2_sync()
+    _check(src.contiguous(), dst.contiguous(), scale)
+    assert bool((out[:, 3] == 0x5A).all()) and bool((out[:, :3, 128:] == 0x5A).all())
+
+
+def test_matches_the_generators_fp8_cache_on_the_1m_workload_rows():
+    wl = inputs.WORKLOADS["c5"].scaled(L=65536)
+    x = inputs.make_inputs(wl.scaled(kv_dtype="bf16"), device=DEV, with_needles=False)
+    q8 = inputs.make_inputs(wl, device=DEV, with_needles=False)
+    dst = torch.empty_like(q8["k"])
+    scale = torch.empty_like(q8["k_scale"])
+    hs2.hs2_quantize_kv(x["k"], dst, scale)
+    hs2.hs2_sync()
+    assert torch.equal(dst, q8["k"]) and torch.equal(scale, q8["k_scale"])   # same bytes as the torch path
+    rows = np.random.default_rng(0).integers(0, 65536, 64)
+    _check(x["k"][rows].cpu(), dst[rows], scale[rows])

@@ -20,6 +20,7 @@
 #include "flash.cuh"
 #include "importance.cuh"
 #include "topk_select.cuh"
+#include "quantize.cuh"
 
 namespace hs2 {
 namespace {
@@ -460,6 +461,34 @@ int hs2_full_attn_select_static(const hs2_shape* shape, const void* q, const voi
   if ((rc = static_scratch(&scratch))) return rc;
   size_t n = kStaticScratchBytes;
   return hs2_full_attn_select(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, scratch, &n, stream);
+}
+
+int hs2_quantize_kv(int32_t L, int32_t Hkv, const void* src, int64_t src_tok_stride, int64_t src_head_stride,
+                    void* dst, int64_t dst_tok_stride, int64_t dst_head_stride, float* scale, void* stream) {
+  if (L <= 0 || Hkv <= 0 || !src || !dst || !scale) return HS2_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(L) * Hkv >= (int64_t(1) << 31)) return HS2_ERR_UNSUPPORTED;
+  if (src_tok_stride <= 0 || src_head_stride <= 0 || dst_tok_stride <= 0 || dst_head_stride <= 0)
+    return HS2_ERR_INVALID_ARG;
+  if (src_head_stride < HD || dst_head_stride < HD || src_tok_stride < static_cast<int64_t>(Hkv) * src_head_stride ||
+      dst_tok_stride < static_cast<int64_t>(Hkv) * dst_head_stride)
+    return HS2_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(src) & 15u) || (reinterpret_cast<uintptr_t>(dst) & 7u) ||
+      (reinterpret_cast<uintptr_t>(scale) & 3u) || src_tok_stride % 8 || src_head_stride % 8 ||
+      dst_tok_stride % 8 || dst_head_stride % 8)
+    return HS2_ERR_UNSUPPORTED;
+  QuantParams p{};
+  p.rows = L * Hkv;
+  p.Hkv = Hkv;
+  p.src = static_cast<const __nv_bfloat16*>(src);
+  p.src_tok = src_tok_stride;
+  p.src_head = src_head_stride;
+  p.dst = static_cast<uint8_t*>(dst);
+  p.dst_tok = dst_tok_stride;
+  p.dst_head = dst_head_stride;
+  p.scale = scale;
+  const int64_t blocks = std::min<int64_t>((static_cast<int64_t>(p.rows) + 63) / 64, 148 * 16);
+  quantize_kv_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return launched();
 }
 
 int hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,

@@ -21,7 +21,7 @@ HS2_KV_BF16, HS2_KV_E4M3 = 0, 1
 
 EXPORTS = ("hs2_full_attn_select", "hs2_sparse_attn", "hs2_sync", "hs2_attn_fwd", "hs2_importance",
            "hs2_topk_select", "hs2_strerror", "hs2_debug_set", "hs2_version", "hs2_launch_count",
-           "hs2_full_attn_select_static", "hs2_exp2_check")
+           "hs2_full_attn_select_static", "hs2_exp2_check", "hs2_quantize_kv")
 
 
 class Hs2Shape(ctypes.Structure):
@@ -51,6 +51,7 @@ _SIGS = {
     "hs2_topk_select": [ctypes.POINTER(Hs2Shape), _vp, _i64, _i32, _i32, _vp, _vp, _vp],
     "hs2_debug_set": [_u64, _u32],
     "hs2_exp2_check": [_vp, _vp, _vp, _vp, _i64, _vp],
+    "hs2_quantize_kv": [_i32, _i32, _vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp],
     "hs2_version": [],
 }
 
@@ -142,6 +143,13 @@ def hs2_importance(shape, q, k, k_scale, lse, b0, b1, imp, row_stride, stream=No
 def hs2_topk_select(shape, imp, row_stride, b0, b1, idx, cnt, stream=None) -> None:
     _check(lib().hs2_topk_select(ctypes.byref(shape), _ptr(imp), int(row_stride), int(b0), int(b1), _ptr(idx),
                                  _ptr(cnt), _stream(stream)), "hs2_topk_select")
+
+
+def hs2_quantize_kv(src, dst, scale, stream=None) -> None:
+    """bf16 [L][Hkv][128] -> e4m3 codes (uint8, same shape) + fp32 scales [L][Hkv]."""
+    L, Hkv, _ = src.shape
+    _check(lib().hs2_quantize_kv(int(L), int(Hkv), _ptr(src), src.stride(0), src.stride(1), _ptr(dst), dst.stride(0),
+                                 dst.stride(1), _ptr(scale), _stream(stream)), "hs2_quantize_kv")
 
 
 def hs2_sync(stream=None) -> None:

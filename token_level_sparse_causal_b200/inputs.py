@@ -141,7 +141,9 @@ def quantize_e4m3(x: torch.Tensor) -> tuple:
     +-448 so nothing overflows to NaN.  Returns (uint8 codes, fp32 scales)."""
     xf = x.float()
     amax = xf.abs().amax(dim=-1)
-    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    # tensor / tensor: an IEEE fp32 division (torch turns division by a Python
+    # scalar into a multiply by its reciprocal, which can differ in the last bit)
+    scale = torch.where(amax > 0, amax / torch.full_like(amax, E4M3_MAX), torch.ones_like(amax))
     y = (xf / scale[..., None]).clamp_(-E4M3_MAX, E4M3_MAX)
     codes = y.to(torch.float8_e4m3fn).view(torch.uint8)
     return codes.contiguous(), scale.contiguous()
