@@ -432,3 +432,59 @@ def test_quantize_kv_row_definition():
     assert np.all(np.abs(deq - x) <= np.abs(x) * 2.0 ** -4 + scale[..., None] * 2.0 ** -9 + 1e-12)
     top = np.abs(x).argmax(axis=-1)
     assert np.all(np.abs(np.take_along_axis(orc.decode_e4m3(codes), top[..., None], -1)[..., 0][nz]) == 448.0)
+
+
+# ------------------------------------------------ block-level selection (v1) --
+
+def test_pool_blocks_tree_is_a_sum():
+    rng = np.random.default_rng(9)
+    I = rng.random(64 * 37).astype(np.float32)
+    J = orc.pool_blocks_fp32(I)
+    ref = I.astype(np.float64).reshape(-1, 64).sum(axis=1)
+    assert J.dtype == np.float32 and np.all(np.abs(J - ref) <= 64 * 2.0 ** -24 * ref)
+    Iz = np.zeros(64 * 3, np.float32)
+    Iz[64 + 7] = 3.0                                   # exact in any order
+    assert list(orc.pool_blocks_fp32(Iz)) == [0.0, 3.0, 0.0]
+
+
+def check_select_blocks_brute(sel_fn, seed=0):
+    """Brute force at block granularity: block m is kept iff fewer than k/64
+    blocks beat it (higher pooled value, or equal and lower index)."""
+    rng = np.random.default_rng(seed)
+    k, w, B = 256, 128, 64
+    bad = 0
+    for L in (128, 192, 512, 1024, 2048):
+        for b in range(L // B):
+            e_b = B * (b + 1)
+            n_c = orc.n_candidates(e_b, w)
+            I = (rng.integers(0, 3, n_c) / 2.0).astype(np.float32)
+            idx, cnt = sel_fn(I, k, w, e_b)
+            J = orc.pool_blocks_fp32(I).astype(np.float64) if n_c else np.zeros(0)
+            rank = orc.brute_rank(J)
+            want = [p for m in range(J.size) if rank[m] < k // B for p in range(m * B, (m + 1) * B)]
+            want += list(range(max(0, e_b - w), e_b))
+            bad += int(list(idx[:cnt]) != want) + int(np.any(idx[cnt:] != -1))
+    return bad
+
+
+def test_select_blocks_brute_force_and_sizes():
+    for seed in range(3):
+        assert check_select_blocks_brute(orc.select_blocks, seed) == 0
+    e_b = 4096
+    idx, cnt = orc.select_blocks(np.ones(e_b - 128, np.float32), 1024, 128, e_b)
+    assert cnt == 1152 and np.array_equal(idx[:1024], np.arange(1024))          # ties -> lowest blocks
+    assert cnt == orc.list_size(e_b, 1024, 128)
+
+
+def test_select_blocks_planted_mistake_is_caught():
+    def ties_high(I, k, w, e_b, B=64):
+        n_c = orc.n_candidates(e_b, w)
+        J = orc.pool_blocks_fp32(np.asarray(I, np.float32)).astype(np.float64) if n_c else np.zeros(0)
+        m = np.arange(J.size)
+        keep = np.sort(np.lexsort((-m, -J))[:min(J.size, k // B)])
+        top = (keep[:, None] * B + np.arange(B)[None, :]).reshape(-1)
+        ch = np.concatenate([top, np.arange(max(0, e_b - w), e_b)])
+        idx = np.full(k + w, -1, np.int64)
+        idx[:ch.size] = ch
+        return idx, ch.size
+    assert check_select_blocks_brute(ties_high) > 0
