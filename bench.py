@@ -343,6 +343,9 @@ def run_cuda(args, wl, rank, world, dist):
                                               o_sp[0], stream), n_stage) if o_sp else 0.0
     fs_ms = timed(lambda: hs2.hs2_full_attn_select(shape, q0, k, v, None, None, out["o"], out["lse"], out["idx"],
                                                    out["cnt"], out["workspace"], stream), n_stage)
+    blk_ms = timed(lambda: hs2.hs2_full_attn_select_blocks(shape, q0, k, v, None, None, out["o"], out["lse"],
+                                                           out["idx"], out["cnt"], out["workspace"], stream),
+                   n_stage) if wl.topk % 64 == 0 and k.dtype == torch.bfloat16 else None
     hs2.hs2_sync(stream)
 
     # ---- end to end from pinned host buffers through the same C ABI calls
@@ -410,7 +413,9 @@ def run_cuda(args, wl, rank, world, dist):
                                        (peaks["bf16_tflops_sustained"] * 1e12) +
                                        2 * work["select_bytes"] / (peaks["hbm_gbs"] * 1e9)),
         },
-        "next_rows": {"fp8_kv_write_K": fp8},
+        "next_rows": {"fp8_kv_write_K": fp8,
+                      "block_level_full_attn_select_ms": blk_ms,
+                      "token_level_full_attn_select_ms": fs_ms},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "e2e": e2e,

@@ -183,6 +183,26 @@ int hs2_importance(const hs2_shape* shape, const void* q, const void* k, const f
 int hs2_topk_select(const hs2_shape* shape, const float* imp, int64_t row_stride, int32_t b0, int32_t b1,
                     int32_t* idx, int32_t* cnt, void* stream);
 
+/* ---- block-level selection (HySparse v1), the design token-level replaces ---- */
+
+/*
+ * Like hs2_topk_select, at the granularity of the earlier HySparse (HySparse2
+ * architecture summary, block-selection paragraph: a whole 64-token block
+ * spends budget): each candidate row is pooled into 64-key blocks -- the sum
+ * of a block in a fixed fp32 order: 16 partial sums of 4 consecutive values
+ * added left to right, then combined pairwise at distances 8, 4, 2, 1 -- the
+ * top topk/64 blocks are kept (ties to the lower block) and listed as
+ * ascending positions, followed by the recent window.  Same layouts and list
+ * sizes as the token-level lists.  Requires topk % 64 == 0.
+ */
+int hs2_block_select(const hs2_shape* shape, const float* imp, int64_t row_stride, int32_t b0, int32_t b1,
+                     int32_t* idx, int32_t* cnt, void* stream);
+
+/* hs2_full_attn_select with block-level instead of token-level selection. */
+int hs2_full_attn_select_blocks(const hs2_shape* shape, const void* q, const void* k, const void* v,
+                                const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,
+                                int32_t* cnt, void* workspace, size_t* workspace_bytes, void* stream);
+
 /* ---- diagnostics ---- */
 
 /* Short text for an hs2_status code (static storage). */

@@ -23,7 +23,8 @@ def lib():
 
 
 def _declared():
-    text = open(os.path.join(ROOT, "include", "hs2.h")).read()
+    with open(os.path.join(ROOT, "include", "hs2.h")) as f:
+        text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(hs2_[a-z_0-9]+)\s*\(", text)))
 
@@ -152,3 +153,14 @@ def test_quantize_kv_argument_checks(lib):
     assert lib.hs2_quantize_kv(16, 2, ctypes.c_void_p(0x10008), 256, 128, P, 256, 128, P, st) == \
         hs2.HS2_ERR_UNSUPPORTED
     assert lib.hs2_quantize_kv(16, 2, P, 256, 128, P, 260, 128, P, st) == hs2.HS2_ERR_UNSUPPORTED
+
+
+def test_block_select_needs_topk_multiple_of_64(lib):
+    s = ctypes.byref(_shape(topk=1000))
+    st = ctypes.c_void_p(0)
+    assert lib.hs2_block_select(s, P, 4096, 0, 1, P, P, st) == hs2.HS2_ERR_UNSUPPORTED
+    n = ctypes.c_size_t(1 << 30)
+    assert lib.hs2_full_attn_select_blocks(s, P, P, P, None, None, P, P, P, P, P, ctypes.byref(n), st) == \
+        hs2.HS2_ERR_UNSUPPORTED
+    s2 = ctypes.byref(_shape())
+    assert lib.hs2_block_select(s2, None, 4096, 0, 1, P, P, st) == hs2.HS2_ERR_INVALID_ARG

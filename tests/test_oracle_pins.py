@@ -119,7 +119,8 @@ def test_dense_invariants():
 
 
 def test_handworked_golden(golden_dir):
-    gd = json.load(open(os.path.join(golden_dir, "handworked_attention.json")))
+    with open(os.path.join(golden_dir, "handworked_attention.json")) as f:
+        gd = json.load(f)
     num = lambda x: math.log(3) if x == "ln3" else (math.log(4) if x == "ln4" else float(x))
     Q = np.array([[[num(x) for x in r]] for r in gd["q"]])
     K = np.array([[[num(x) for x in r]] for r in gd["k"]])
@@ -228,7 +229,8 @@ def test_select_all_equal_takes_first_positions():
 
 
 def test_select_invariants_and_golden_sizes(golden_dir):
-    gd = json.load(open(os.path.join(golden_dir, "list_sizes_L2048.json")))
+    with open(os.path.join(golden_dir, "list_sizes_L2048.json")) as f:
+        gd = json.load(f)
     L, B, k, w = gd["L"], gd["block"], gd["topk"], gd["recent"]
     rng = np.random.default_rng(3)
     for b in range(L // B):

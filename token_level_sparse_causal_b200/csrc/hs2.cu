@@ -266,7 +266,7 @@ int launch_importance(const hs2_shape* s, const void* q, const void* k, const fl
 }
 
 int launch_select(const hs2_shape* s, const float* imp, int64_t row_stride, int b0, int b1, int32_t* idx,
-                  int32_t* cnt, cudaStream_t st) {
+                  int32_t* cnt, cudaStream_t st, bool blocks = false) {
   SelParams p{};
   p.L = s->L;
   p.Hkv = s->Hkv;
@@ -280,7 +280,15 @@ int launch_select(const hs2_shape* s, const float* imp, int64_t row_stride, int 
   p.row_stride = row_stride;
   p.idx = idx;
   p.cnt = cnt;
-  topk_select_kernel<<<static_cast<unsigned>(s->Hkv * (b1 - b0)), SEL_THREADS, 0, st>>>(p);
+  const unsigned grid = static_cast<unsigned>(s->Hkv * (b1 - b0));
+  if (blocks) {
+    const uint32_t dyn = static_cast<uint32_t>(s->L / 64) * 4u;  // pooled values of the longest row
+    static int attr = set_smem(block_select_kernel, 64u * 1024u);
+    if (attr) return attr;
+    block_select_kernel<<<grid, SEL_THREADS, dyn, st>>>(p);
+  } else {
+    topk_select_kernel<<<grid, SEL_THREADS, 0, st>>>(p);
+  }
   return launched();
 }
 
@@ -411,9 +419,54 @@ int hs2_topk_select(const hs2_shape* shape, const float* imp, int64_t row_stride
   return launch_select(shape, imp, row_stride, b0, b1, idx, cnt, static_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+namespace hs2 {
+namespace {
+int full_attn_select_impl(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
+                          const float* v_scale, void* o, float* lse, int32_t* idx, int32_t* cnt, void* workspace,
+                          size_t* workspace_bytes, void* stream, bool blocks);
+}  // namespace
+}  // namespace hs2
+
+extern "C" {
+
 int hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
                          const float* v_scale, void* o, float* lse, int32_t* idx, int32_t* cnt, void* workspace,
                          size_t* workspace_bytes, void* stream) {
+  return full_attn_select_impl(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, workspace, workspace_bytes, stream,
+                               false);
+}
+
+int hs2_full_attn_select_blocks(const hs2_shape* shape, const void* q, const void* k, const void* v,
+                                const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,
+                                int32_t* cnt, void* workspace, size_t* workspace_bytes, void* stream) {
+  if (shape && shape->topk % 64) return HS2_ERR_UNSUPPORTED;
+  return full_attn_select_impl(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, workspace, workspace_bytes, stream,
+                               true);
+}
+
+int hs2_block_select(const hs2_shape* shape, const float* imp, int64_t row_stride, int32_t b0, int32_t b1,
+                     int32_t* idx, int32_t* cnt, void* stream) {
+  using namespace hs2;
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (shape->topk % 64) return HS2_ERR_UNSUPPORTED;
+  if (!imp || !idx || !cnt) return HS2_ERR_INVALID_ARG;
+  const int nb = shape->L / 64;
+  if (b0 < 0 || b1 > nb || b0 >= b1) return HS2_ERR_INVALID_ARG;
+  if (row_stride % 4 || row_stride < n_cand(shape, b1 - 1)) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(imp)) return HS2_ERR_UNSUPPORTED;
+  return launch_select(shape, imp, row_stride, b0, b1, idx, cnt, static_cast<cudaStream_t>(stream), true);
+}
+
+}  // extern "C"
+
+namespace hs2 {
+namespace {
+int full_attn_select_impl(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
+                          const float* v_scale, void* o, float* lse, int32_t* idx, int32_t* cnt, void* workspace,
+                          size_t* workspace_bytes, void* stream, bool blocks) {
   int rc = check_shape(shape);
   if (rc) return rc;
   if (!workspace_bytes) return HS2_ERR_INVALID_ARG;
@@ -444,12 +497,16 @@ int hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, c
       while (b1 < nb && static_cast<size_t>(shape->Hkv) * (b1 + 1 - b) * strip_stride(shape, b1) * 4u <= ws) ++b1;
       const int64_t stride = strip_stride(shape, b1 - 1);
       if ((rc = launch_importance(shape, q, k, k_scale, lse, b, b1, imp, stride, shape->topk, st))) return rc;
-      if ((rc = launch_select(shape, imp, stride, b, b1, idx, cnt, st))) return rc;
+      if ((rc = launch_select(shape, imp, stride, b, b1, idx, cnt, st, blocks))) return rc;
     }
     b = b1;
   }
   return HS2_OK;
 }
+}  // namespace
+}  // namespace hs2
+
+extern "C" {
 
 int hs2_full_attn_select_static(const hs2_shape* shape, const void* q, const void* k, const void* v,
                                 const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,

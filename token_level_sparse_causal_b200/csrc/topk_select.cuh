@@ -175,4 +175,109 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelParam
   if (tid == 0) p.cnt[static_cast<int64_t>(g) * p.nb + b] = total;
 }
 
+// Block-level selection (HySparse v1, the design the token-level selection
+// replaces; HySparse2 architecture summary, block-selection paragraph): each
+// candidate row is pooled into 64-key blocks, the top topk/64 blocks by pooled
+// importance are kept (ties to the lower block) and expanded to positions.
+// The pooled sum of a block is defined in a fixed fp32 order: 16 lanes each
+// add 4 consecutive values left to right, then a butterfly over the 16 lanes
+// (l ^ 8, ^ 4, ^ 2, ^ 1); every step is commutative, so all lanes hold the
+// same bits.  One 512-thread CTA per row; pooled values live in shared memory.
+__global__ void __launch_bounds__(SEL_THREADS) block_select_kernel(const SelParams p) {
+  extern __shared__ float pooled[];  // [n_blk]
+  __shared__ uint32_t hist[2048];
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t sh_digit, sh_above;
+  __shared__ int sel[64];
+
+  const int y = blockIdx.x;
+  const int g = y / p.nbs;
+  const int b = p.b0 + y % p.nbs;
+  const int e_b = min(p.L, 64 * (b + 1));
+  const int n_c = max(0, e_b - p.recent);
+  const int nrec = min(p.recent, e_b);
+  const int n_blk = n_c / 64, kb = p.topk / 64;
+  const int nsel = min(n_blk, kb);
+  int32_t* list = p.idx + (static_cast<int64_t>(g) * p.nb + b) * p.list_len;
+  const int tid = threadIdx.x;
+
+  if (n_blk > kb) {
+    const float4* row4 = reinterpret_cast<const float4*>(p.imp + (static_cast<int64_t>(g) * p.nbs + (b - p.b0)) *
+                                                                    p.row_stride);
+    const int l16 = tid & 15;
+    // a half-warp per block; the loop bound is warp-uniform (full-mask shuffles)
+    for (int m0 = (tid >> 5) * 2; m0 < n_blk; m0 += SEL_THREADS / 16) {
+      const int m = m0 + ((tid >> 4) & 1);
+      const float4 v = (m < n_blk) ? __ldg(row4 + m * 16 + l16) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float a = ((v.x + v.y) + v.z) + v.w;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) a = a + __shfl_xor_sync(0xffffffffu, a, o);
+      if (m < n_blk && l16 == 0) pooled[m] = a;
+    }
+    __syncthreads();
+    uint32_t prefix = 0, pmask = 0, krem = static_cast<uint32_t>(kb);
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = (pass == 0) ? 21 : (pass == 1) ? 10 : 0;
+      const int nbins = (pass == 2) ? 1024 : 2048;
+      for (int i = tid; i < nbins; i += SEL_THREADS) hist[i] = 0;
+      __syncthreads();
+      for (int m = tid; m < n_blk; m += SEL_THREADS) {
+        const uint32_t key = order_key(pooled[m]);
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nbins - 1)], 1u);
+      }
+      __syncthreads();
+      const int per = nbins / SEL_THREADS;
+      uint32_t loc = 0;
+      for (int q = 0; q < per; ++q) loc += hist[nbins - 1 - (tid * per + q)];
+      uint32_t tot;
+      const uint32_t ex = block_excl_scan(loc, warp_sums, &tot);
+      if (ex < krem && ex + loc >= krem) {
+        uint32_t run = ex;
+        for (int q = 0; q < per; ++q) {
+          const int bin = nbins - 1 - (tid * per + q);
+          const uint32_t c = hist[bin];
+          if (run + c >= krem) {
+            sh_digit = static_cast<uint32_t>(bin);
+            sh_above = run;
+            break;
+          }
+          run += c;
+        }
+      }
+      __syncthreads();
+      prefix |= sh_digit << shift;
+      pmask |= static_cast<uint32_t>(nbins - 1) << shift;
+      krem -= sh_above;
+      __syncthreads();
+    }
+    const uint32_t T = prefix;
+    uint32_t gt_carry = 0, eq_carry = 0;
+#pragma unroll 1
+    for (int base = 0; base < n_blk; base += SEL_THREADS) {
+      const int m = base + tid;
+      bool gt = false, eq = false;
+      if (m < n_blk) {
+        const uint32_t key = order_key(pooled[m]);
+        gt = key > T;
+        eq = key == T;
+      }
+      uint32_t tot;
+      const uint32_t ex = block_excl_scan((gt ? 1u << 16 : 0u) | (eq ? 1u : 0u), warp_sums, &tot);
+      const uint32_t gt_before = gt_carry + (ex >> 16), eq_before = eq_carry + (ex & 0xFFFFu);
+      if (gt) sel[gt_before + min(eq_before, krem)] = m;
+      else if (eq && eq_before < krem) sel[gt_before + eq_before] = m;
+      gt_carry += tot >> 16;
+      eq_carry += tot & 0xFFFFu;
+    }
+  } else {
+    for (int i = tid; i < nsel; i += SEL_THREADS) sel[i] = i;
+  }
+  __syncthreads();
+  for (int i = tid; i < nsel * 64; i += SEL_THREADS) list[i] = sel[i >> 6] * 64 + (i & 63);
+  for (int i = tid; i < nrec; i += SEL_THREADS) list[nsel * 64 + i] = e_b - nrec + i;
+  for (int i = nsel * 64 + nrec + tid; i < p.list_len; i += SEL_THREADS) list[i] = -1;
+  if (tid == 0) p.cnt[static_cast<int64_t>(g) * p.nb + b] = nsel * 64 + nrec;
+}
+
 }  // namespace hs2

@@ -21,7 +21,8 @@ HS2_KV_BF16, HS2_KV_E4M3 = 0, 1
 
 EXPORTS = ("hs2_full_attn_select", "hs2_sparse_attn", "hs2_sync", "hs2_attn_fwd", "hs2_importance",
            "hs2_topk_select", "hs2_strerror", "hs2_debug_set", "hs2_version", "hs2_launch_count",
-           "hs2_full_attn_select_static", "hs2_exp2_check", "hs2_quantize_kv")
+           "hs2_full_attn_select_static", "hs2_exp2_check", "hs2_quantize_kv", "hs2_block_select",
+           "hs2_full_attn_select_blocks")
 
 
 class Hs2Shape(ctypes.Structure):
@@ -44,6 +45,9 @@ _SIGS = {
     "hs2_full_attn_select": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                              ctypes.POINTER(ctypes.c_size_t), _vp],
     "hs2_full_attn_select_static": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "hs2_full_attn_select_blocks": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                    ctypes.POINTER(ctypes.c_size_t), _vp],
+    "hs2_block_select": [ctypes.POINTER(Hs2Shape), _vp, _i64, _i32, _i32, _vp, _vp, _vp],
     "hs2_sparse_attn": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "hs2_sync": [_vp],
     "hs2_attn_fwd": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
@@ -123,6 +127,18 @@ def hs2_full_attn_select_static(shape, q, k, v, k_scale, v_scale, o, lse, idx, c
     _check(lib().hs2_full_attn_select_static(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale),
                                              _ptr(v_scale), _ptr(o), _ptr(lse), _ptr(idx), _ptr(cnt),
                                              _stream(stream)), "hs2_full_attn_select_static")
+
+
+def hs2_full_attn_select_blocks(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, workspace, stream=None) -> None:
+    n = ctypes.c_size_t(workspace.numel() * workspace.element_size())
+    _check(lib().hs2_full_attn_select_blocks(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale),
+                                             _ptr(v_scale), _ptr(o), _ptr(lse), _ptr(idx), _ptr(cnt), _ptr(workspace),
+                                             ctypes.byref(n), _stream(stream)), "hs2_full_attn_select_blocks")
+
+
+def hs2_block_select(shape, imp, row_stride, b0, b1, idx, cnt, stream=None) -> None:
+    _check(lib().hs2_block_select(ctypes.byref(shape), _ptr(imp), int(row_stride), int(b0), int(b1), _ptr(idx),
+                                  _ptr(cnt), _stream(stream)), "hs2_block_select")
 
 
 def hs2_sparse_attn(shape, q, k, v, k_scale, v_scale, idx, cnt, o, stream=None) -> None:
