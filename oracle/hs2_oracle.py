@@ -166,6 +166,31 @@ def dense_attn(Q, K, V, r0: int = 0, r1: int | None = None):
     return O, lse
 
 
+def swa_attn(Q, K, V, W: int):
+    """Causal sliding-window attention: query i attends to keys
+    max(0, i - W + 1) <= j <= i ([HS2] two-part paragraph: the self-decoder
+    combines full and sliding-window attention; the window width is this
+    library's parameter, 128 in the measurements).  Returns O and lse like
+    dense_attn."""
+    L, Hq, d = Q.shape
+    G = Hq // K.shape[1]
+    i = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    visible = (j <= i) & (j > i - W)
+    O = np.empty((L, Hq, d))
+    lse = np.empty((Hq, L))
+    for h in range(Hq):
+        g = kv_head(h, G)
+        s = (Q[:, h, :] @ K[:, g, :].T) / np.sqrt(d)
+        s = np.where(visible, s, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        p = np.exp(s - m)
+        l = p.sum(axis=1, keepdims=True)
+        O[:, h, :] = (p @ V[:, g, :]) / l
+        lse[h] = (m + np.log(l))[:, 0]
+    return O, lse
+
+
 # ------------------------------------------------------------ importance --
 
 

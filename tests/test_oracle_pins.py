@@ -490,3 +490,21 @@ def test_select_blocks_planted_mistake_is_caught():
         idx[:ch.size] = ch
         return idx, ch.size
     assert check_select_blocks_brute(ties_high) > 0
+
+
+# ------------------------------------------------- sliding-window attention --
+
+def test_swa_matches_sdpa_with_band_mask():
+    L, Hq, Hkv, d = 150, 4, 2, 16
+    Q, K, V = _rand((L, Hq, d), 71), _rand((L, Hkv, d), 72), _rand((L, Hkv, d), 73)
+    for W in (1, 7, 64, 128):
+        O, lse = orc.swa_attn(Q, K, V, W)
+        i, j = np.arange(L)[:, None], np.arange(L)[None, :]
+        band = np.broadcast_to((j <= i) & (j > i - W), (Hq, L, L)).copy()
+        assert np.abs(O - _sdpa(Q, K, V, mask=band)).max() < 1e-12
+    O1, _ = orc.swa_attn(Q, K, V, 1)                 # each query sees only itself
+    G = Hq // Hkv
+    assert np.abs(O1 - V[:, np.arange(Hq) // G, :]).max() < 1e-15
+    Ofull, lfull = orc.swa_attn(Q, K, V, L)         # window >= L is plain causal attention
+    Od, ld = orc.dense_attn(Q, K, V)
+    assert np.abs(Ofull - Od).max() < 1e-13 and np.abs(lfull - ld).max() < 1e-13
