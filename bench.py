@@ -37,6 +37,9 @@ METRIC = "prefill tok/s (full-attn+select+sparse-attn) at 128k on 1 B200; % of r
 
 # ------------------------------------------------------------ accounting --
 
+SWA_WINDOW = 128   # sliding window of the self-decoder layers in the measurements
+
+
 def algorithmic_work(wl) -> dict:
     """Exact causal counts of what the method must compute or move."""
     L, Hq, Hkv, d, B, k, w = wl.L, wl.Hq, wl.Hkv, wl.d, wl.block, wl.topk, wl.recent
@@ -55,8 +58,14 @@ def algorithmic_work(wl) -> dict:
     sparse = Hq * 4.0 * d * vis.sum()
     gather = Hkv * (glob + rec).sum() * 2 * 256.0
     qo = 2.0 * L * Hq * d * 2
+    # sliding-window attention: query i sees min(i + 1, W) keys; Q, K, V read
+    # once and O written once
+    W = SWA_WINDOW
+    swa_pairs = W * (W + 1) / 2.0 + max(0, L - W) * float(W) if L >= W else L * (L + 1) / 2.0
+    swa = Hq * 4.0 * d * swa_pairs
+    swa_bytes = qo + 2.0 * L * Hkv * d * 2
     return {"fa_flop": fa, "imp_flop": imp, "select_bytes": select_bytes, "sparse_flop": sparse,
-            "gather_bytes": gather, "sparse_qo_bytes": qo}
+            "gather_bytes": gather, "sparse_qo_bytes": qo, "swa_flop": swa, "swa_bytes": swa_bytes}
 
 
 FA_SOURCES = ("token_level_sparse_causal_b200/csrc/flash.cuh", "token_level_sparse_causal_b200/csrc/common.cuh")
@@ -346,6 +355,8 @@ def run_cuda(args, wl, rank, world, dist):
     blk_ms = timed(lambda: hs2.hs2_full_attn_select_blocks(shape, q0, k, v, None, None, out["o"], out["lse"],
                                                            out["idx"], out["cnt"], out["workspace"], stream),
                    n_stage) if wl.topk % 64 == 0 and k.dtype == torch.bfloat16 else None
+    swa_ms = timed(lambda: hs2.hs2_swa_attn(shape, q0, k, v, SWA_WINDOW, out["o"], None, stream),
+                   n_stage) if k.dtype == torch.bfloat16 else None
     hs2.hs2_sync(stream)
 
     # ---- end to end from pinned host buffers through the same C ABI calls
@@ -415,7 +426,16 @@ def run_cuda(args, wl, rank, world, dist):
         },
         "next_rows": {"fp8_kv_write_K": fp8,
                       "block_level_full_attn_select_ms": blk_ms,
-                      "token_level_full_attn_select_ms": fs_ms},
+                      "token_level_full_attn_select_ms": fs_ms,
+                      "swa_attn": None if swa_ms is None else {
+                          "window": SWA_WINDOW, "ms": swa_ms,
+                          "tflops": work["swa_flop"] / (swa_ms / 1e3) / 1e12,
+                          "gbs": work["swa_bytes"] / (swa_ms / 1e3) / 1e9,
+                          "roofline_ms": 1e3 * max(work["swa_flop"] / (peaks["bf16_tflops"] * 1e12),
+                                                   work["swa_bytes"] / (peaks["hbm_gbs"] * 1e9)),
+                          "frac_of_roofline": 1e3 * max(work["swa_flop"] / (peaks["bf16_tflops"] * 1e12),
+                                                        work["swa_bytes"] / (peaks["hbm_gbs"] * 1e9)) / swa_ms,
+                      }},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "e2e": e2e,

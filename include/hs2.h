@@ -203,6 +203,23 @@ int hs2_full_attn_select_blocks(const hs2_shape* shape, const void* q, const voi
                                 const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,
                                 int32_t* cnt, void* workspace, size_t* workspace_bytes, void* stream);
 
+/* ---- sliding-window attention (self-decoder window layers) ---- */
+
+/*
+ * Causal sliding-window attention: o_i = softmax over j in (i - window, i] of
+ * q_i . k_j / sqrt(d), applied to v (HySparse2 architecture summary, paragraph
+ * on the self-decoder / cross-decoder split: the front half mixes full and
+ * sliding-window attention).  Same q / k / v / o layouts and strides as
+ * hs2_attn_fwd; the cache must be bf16 (kv_dtype = HS2_KV_BF16, else
+ * HS2_ERR_UNSUPPORTED); topk / recent are checked as in every call but not
+ * used.  1 <= window <= L, else HS2_ERR_INVALID_ARG.  lse (fp32 [Hq][L],
+ * natural log) is optional: NULL skips it, otherwise it must be 16-byte
+ * aligned.  Device pointers owned by the caller; asynchronous on `stream`;
+ * device-side failures surface through hs2_sync.
+ */
+int hs2_swa_attn(const hs2_shape* shape, const void* q, const void* k, const void* v, int32_t window, void* o,
+                 float* lse, void* stream);
+
 /* ---- diagnostics ---- */
 
 /* Short text for an hs2_status code (static storage). */

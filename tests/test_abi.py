@@ -164,3 +164,17 @@ def test_block_select_needs_topk_multiple_of_64(lib):
         hs2.HS2_ERR_UNSUPPORTED
     s2 = ctypes.byref(_shape())
     assert lib.hs2_block_select(s2, None, 4096, 0, 1, P, P, st) == hs2.HS2_ERR_INVALID_ARG
+
+
+def test_swa_argument_checks(lib):
+    st = ctypes.c_void_p(0)
+    s = ctypes.byref(_shape())
+    assert lib.hs2_swa_attn(s, P, P, P, 0, P, None, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_swa_attn(s, P, P, P, 2049, P, None, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_swa_attn(s, None, P, P, 128, P, None, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_swa_attn(s, P, P, P, 128, None, None, st) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_swa_attn(s, P, P, P, 128, P, MIS, st) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_swa_attn(s, MIS, P, P, 128, P, None, st) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_swa_attn(ctypes.byref(_shape(kv_dtype=1)), P, P, P, 128, P, None, st) == \
+        hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_swa_attn(ctypes.byref(_shape(d=64)), P, P, P, 128, P, None, st) == hs2.HS2_ERR_UNSUPPORTED

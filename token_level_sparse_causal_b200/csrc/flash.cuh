@@ -15,6 +15,12 @@
 //                   rows are gathered with 16-byte cp.async into swizzled
 //                   shared memory; the causal mask j <= i applies to listed
 //                   positions.
+//   FLASH_SWA    -- causal sliding-window attention of the self-decoder's
+//                   window layers (HySparse2 architecture summary, paragraph
+//                   on the self-decoder / cross-decoder split): the dense
+//                   pipeline with query tile x starting at key tile lo(x),
+//                   the first one that meets the window, and a band mask
+//                   i - window < j <= i.  bf16 cache only.
 //
 // CTA = 12 warps:
 //   warp 0      TMA: Q tiles (both modes), K/V tiles (dense)
@@ -63,6 +69,7 @@ constexpr uint32_t IDESC_S_F16 = idesc_f16_f32(128, 128, 0, 0);
 constexpr uint32_t IDESC_PV_F16 = idesc_f16_f32(128, 128, 0, 1);
 constexpr int FLASH_DENSE = 0;
 constexpr int FLASH_SPARSE = 1;
+constexpr int FLASH_SWA = 2;
 constexpr uint32_t FLAG_SKIP_LOADS = 1u;
 constexpr int MAX_LIST = 4096;
 
@@ -71,6 +78,7 @@ struct FlashParams {
   int nb, list_len, mtiles, rows_tok;  // sparse: blocks, list stride, M tiles per (b,g), tokens per M tile
   int mpairs;                          // sparse: pairs of M tiles per (b,g)
   float scale_log2;                    // log2(e) / sqrt(d)
+  int window;                          // SWA: keys i - window < j <= i
   const __nv_bfloat16* k;              // gather sources (sparse)
   const __nv_bfloat16* v;
   const uint8_t* k8;                   // e4m3 codes and fp32 scales [L][Hkv] (KV8)
@@ -137,6 +145,7 @@ template <int MODE, bool KV8>
 __global__ void __launch_bounds__(FL_THREADS, 1)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const FlashParams p) {
+  static_assert(!(MODE == FLASH_SWA && KV8), "the window mode reads a bf16 cache");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   FlashBars* bars = reinterpret_cast<FlashBars*>(smem + FL_BAR_OFF);
@@ -147,9 +156,12 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &bars->abort;
 
-  // ---- work item: query tiles A and B (B may be absent), key tiles nA / nB
+  // ---- work item: query tiles A and B (B may be absent); query tile x uses
+  // key tiles lo(x) .. (x ? nB : nA) - 1 (lo is 0 except in SWA mode)
+  constexpr bool kDenseLike = MODE != FLASH_SPARSE;
   int h = 0, g = 0, b = 0, pair = 0, cnt = 0, e_b = 0, nA = 0, nB = 0;
-  if (MODE == FLASH_DENSE) {
+  int lo0 = 0, lo1 = 0;  // first key tile of query tile A / B
+  if (kDenseLike) {
     // KV-group-major order, longest tile pairs first within a group: the
     // CTAs resident at any time share one group's K/V, which then stays in L2.
     const int per_g = p.npairs * p.G;
@@ -159,6 +171,10 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     h = g * p.G + rem % p.G;
     nA = 2 * pair + 1;
     nB = (2 * pair + 1 < p.nqt) ? 2 * pair + 2 : 0;
+    if (MODE == FLASH_SWA) {
+      lo0 = max(0, 2 * pair * 128 - p.window + 1) / 128;
+      lo1 = max(0, (2 * pair + 1) * 128 - p.window + 1) / 128;
+    }
   } else {
     pair = static_cast<int>(blockIdx.x) % p.mpairs;
     const int bg = static_cast<int>(blockIdx.x) / p.mpairs;
@@ -174,10 +190,13 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     for (int i = threadIdx.x; i < nt * 128; i += blockDim.x) pos_s[i] = (i < cnt) ? list[i] : -1;
   }
   const int n = max(nA, nB);
-  const bool has_b = (MODE == FLASH_DENSE) ? (nB > 0) : (2 * pair + 1 < p.mtiles);
+  const int j0 = lo0;  // first key tile of the CTA (lo0 <= lo1)
+  // a compile-time 0 outside SWA mode
+  auto lo = [&](int x) { return MODE == FLASH_SWA ? (x ? lo1 : lo0) : 0; };
+  const bool has_b = kDenseLike ? (nB > 0) : (2 * pair + 1 < p.mtiles);
 
   if (threadIdx.x == 0) {
-    const uint32_t kv_arrivals = (MODE == FLASH_DENSE && !KV8) ? 1u : 64u;
+    const uint32_t kv_arrivals = (kDenseLike && !KV8) ? 1u : 64u;
     mbar_init(&bars->q_raw, 1);
     mbar_init(&bars->q_full, KV8 ? 64u : 1u);
     for (int s = 0; s < FL_STAGES; ++s) {
@@ -212,7 +231,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       mbar_arrive_expect_tx(qbar, static_cast<uint32_t>(nq) * TILE_BYTES);
       for (int x = 0; x < nq; ++x) {
         uint8_t* qd = smem + FL_Q_OFF + x * TILE_BYTES;
-        if (MODE == FLASH_DENSE) {
+        if (kDenseLike) {
           tma_load_3d(qd, &tmQ, qbar, 0, h, (2 * pair + x) * 128);
           tma_load_3d(qd + HALF_BYTES, &tmQ, qbar, 64, h, (2 * pair + x) * 128);
         } else {
@@ -221,12 +240,13 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           tma_load_3d(qd + HALF_BYTES, &tmQ, qbar, 64, g * p.G, t0);
         }
       }
-      if (MODE == FLASH_DENSE && !KV8) {
+      if (kDenseLike && !KV8) {
         int last = -1;
-        for (int j = 0; j < n; ++j) {
-          const int s = j % FL_STAGES;
-          if (j >= FL_STAGES &&
-              !mbar_wait(&bars->empty[s], ((j / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 101))
+        for (int j = j0; j < n; ++j) {
+          const int u = j - j0;  // position in this CTA's key-tile stream
+          const int s = u % FL_STAGES;
+          if (u >= FL_STAGES &&
+              !mbar_wait(&bars->empty[s], ((u / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 101))
             break;
           uint8_t* kd = smem + FL_KV_OFF + s * 2 * TILE_BYTES;
           mbar_arrive_expect_tx(&bars->full_k[s], TILE_BYTES);
@@ -235,13 +255,13 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           mbar_arrive_expect_tx(&bars->full_v[s], TILE_BYTES);
           tma_load_3d(kd + TILE_BYTES, &tmV, &bars->full_v[s], 0, g, j * 128);
           tma_load_3d(kd + TILE_BYTES + HALF_BYTES, &tmV, &bars->full_v[s], 64, g, j * 128);
-          last = j;
+          last = u;
         }
         // Never leave a TMA write in flight into memory the CTA gives back.
-        for (int j = max(0, last - FL_STAGES + 1); j <= last; ++j) {
-          const int s = j % FL_STAGES;
-          wait_done(&bars->full_k[s], (j / FL_STAGES) & 1, p.limit_ns, 102);
-          wait_done(&bars->full_v[s], (j / FL_STAGES) & 1, p.limit_ns, 103);
+        for (int u = max(0, last - FL_STAGES + 1); u <= last; ++u) {
+          const int s = u % FL_STAGES;
+          wait_done(&bars->full_k[s], (u / FL_STAGES) & 1, p.limit_ns, 102);
+          wait_done(&bars->full_v[s], (u / FL_STAGES) & 1, p.limit_ns, 103);
         }
       }
       wait_done(qbar, 0, p.limit_ns, 104);
@@ -251,7 +271,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     if (lane == 0 && n > 0) {
       const int nx[2] = {nA, nB};
       auto issue_s = [&](int x, int j) {
-        const uint32_t kb = kv_base + (j % FL_STAGES) * 2 * TILE_BYTES;
+        const uint32_t kb = kv_base + ((j - j0) % FL_STAGES) * 2 * TILE_BYTES;
         const uint32_t qb = q_base + x * TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -262,12 +282,12 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         umma_commit(&bars->s_full[x]);
       };
       auto issue_pv = [&](int x, int j) {
-        const uint32_t vb = kv_base + (j % FL_STAGES) * 2 * TILE_BYTES + TILE_BYTES;
+        const uint32_t vb = kv_base + ((j - j0) % FL_STAGES) * 2 * TILE_BYTES + TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bdesc = sdesc_sw128(vb + kk * 2048, HALF_BYTES, 1024);
           umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bdesc, KV8 ? IDESC_PV_F16 : IDESC_PV,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+                  (j > lo(x) || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars->o_done[x]);
       };
@@ -276,19 +296,20 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       if (ok) {
         tc_fence_after();
         for (int x = 0; x < 2; ++x)
-          if (nx[x] > 0) issue_s(x, 0);
+          if (nx[x] > lo(x) && lo(x) == j0) issue_s(x, j0);
       }
-      for (int j = 0; j < n && ok; ++j) {
-        const int s = j % FL_STAGES;
+      for (int j = j0; j < n && ok; ++j) {
+        const int u = j - j0;
+        const int s = u % FL_STAGES;
         bool v_ready = false, k_next = false;
         for (int x = 0; x < 2 && ok; ++x) {
-          if (j >= nx[x]) continue;
-          if (!mbar_wait(&bars->p_ready[x], j & 1, p.limit_ns, abort_flag, 113)) {
+          if (j < lo(x) || j >= nx[x]) continue;
+          if (!mbar_wait(&bars->p_ready[x], (j - lo(x)) & 1, p.limit_ns, abort_flag, 113)) {
             ok = false;
             break;
           }
           if (!v_ready) {
-            if (!mbar_wait(&bars->full_v[s], (j / FL_STAGES) & 1, p.limit_ns, abort_flag, 114)) {
+            if (!mbar_wait(&bars->full_v[s], (u / FL_STAGES) & 1, p.limit_ns, abort_flag, 114)) {
               ok = false;
               break;
             }
@@ -298,8 +319,23 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           issue_pv(x, j);
           if (j + 1 < nx[x]) {
             if (!k_next) {
-              const int s1 = (j + 1) % FL_STAGES;
-              if (!mbar_wait(&bars->full_k[s1], ((j + 1) / FL_STAGES) & 1, p.limit_ns, abort_flag, 115)) {
+              const int s1 = (u + 1) % FL_STAGES;
+              if (!mbar_wait(&bars->full_k[s1], ((u + 1) / FL_STAGES) & 1, p.limit_ns, abort_flag, 115)) {
+                ok = false;
+                break;
+              }
+              k_next = true;
+              tc_fence_after();
+            }
+            issue_s(x, j + 1);
+          }
+        }
+        // a query tile whose first key tile is the next one starts now
+        for (int x = 0; x < 2 && ok && MODE == FLASH_SWA; ++x) {
+          if (lo(x) == j + 1 && j + 1 < nx[x]) {
+            if (!k_next) {
+              const int s1 = (u + 1) % FL_STAGES;
+              if (!mbar_wait(&bars->full_k[s1], ((u + 1) / FL_STAGES) & 1, p.limit_ns, abort_flag, 116)) {
                 ok = false;
                 break;
               }
@@ -440,7 +476,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     const uint32_t s_tm = tmem + lane_off + x * 128;
     const uint32_t o_tm = tmem + lane_off + 256 + x * 128;
     int i_row, hh, i_min, diag = -1;
-    if (MODE == FLASH_DENSE) {
+    if (kDenseLike) {
       const int qt = 2 * pair + x;
       i_row = qt * 128 + r;
       hh = h;
@@ -455,8 +491,9 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     const float sc = KV8 ? 1.f : p.scale_log2;  // KV8 folds the scale into the columns
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nX; ++j) {
-      if (!warp_wait(&bars->s_full[x], j & 1, p.limit_ns, abort_flag, 131)) {
+    for (int j = lo(x); j < nX; ++j) {
+      const int t = j - lo(x);  // tiles this query tile has seen before j
+      if (!warp_wait(&bars->s_full[x], t & 1, p.limit_ns, abort_flag, 131)) {
         ok = false;
         break;
       }
@@ -490,6 +527,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       bool need_mask;
       if (MODE == FLASH_DENSE) {
         need_mask = (j == diag);
+      } else if (MODE == FLASH_SWA) {  // the diagonal, or keys below some row's window
+        need_mask = (j == diag) || (j * 128 < i_min + 128 - p.window);
       } else {
         const int last = j * 128 + 127;
         need_mask = (last >= cnt) || (pos_s[last] > i_min);
@@ -499,6 +538,11 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c > r) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+        } else if (MODE == FLASH_SWA) {  // keep i - window < j*128 + c <= i
+          const int c_hi = i_row - j * 128, c_lo = c_hi - p.window;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > c_hi || c <= c_lo) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
         } else {
           const int4* pv4 = reinterpret_cast<const int4*>(pos_s + j * 128);
 #pragma unroll
@@ -561,8 +605,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         l += (a0 + a1) + (b0 + b1);
       }
       // ---- O rescale (needs PV(j-1) complete)
-      if (j > 0) {
-        if (!warp_wait(&bars->o_done[x], (j - 1) & 1, p.limit_ns, abort_flag, 132)) {
+      if (t > 0) {
+        if (!warp_wait(&bars->o_done[x], (t - 1) & 1, p.limit_ns, abort_flag, 132)) {
           ok = false;
           break;
         }
@@ -587,7 +631,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     // ---- epilogue
     const bool row_live = i_row < p.L && (x == 0 || has_b);  // a last dense tile may hang past L
     __nv_bfloat16* orow = p.o + static_cast<int64_t>(i_row) * p.o_tok + static_cast<int64_t>(hh) * p.o_head;
-    if (ok && nX > 0 && warp_wait(&bars->o_done[x], (nX - 1) & 1, p.limit_ns, abort_flag, 133)) {
+    const int nT = nX - lo(x);  // key tiles of this query tile
+    if (ok && nT > 0 && warp_wait(&bars->o_done[x], (nT - 1) & 1, p.limit_ns, abort_flag, 133)) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
@@ -607,7 +652,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
             dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
       }
-      if (MODE == FLASH_DENSE && row_live)
+      if (kDenseLike && row_live && (MODE == FLASH_DENSE || p.lse != nullptr))
         p.lse[static_cast<int64_t>(hh) * p.L + i_row] = (m_used + log2f(l)) * 0.69314718055994530942f;
     } else if (MODE == FLASH_SPARSE && ok && n == 0 && row_live) {
       // an empty list: the rows attend to nothing

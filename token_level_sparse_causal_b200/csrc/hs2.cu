@@ -117,8 +117,9 @@ int set_smem(K kernel, uint32_t bytes) {
 
 // ------------------------------------------------------------- launches --
 
+// window > 0 launches the sliding-window mode (bf16 cache only).
 int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void* v, const float* ks,
-                    const float* vs, void* o, float* lse, cudaStream_t st) {
+                    const float* vs, void* o, float* lse, cudaStream_t st, int window = 0) {
   const bool kv8 = s->kv_dtype == HS2_KV_E4M3;
   CUtensorMap mq, mk, mv;
   int rc;
@@ -150,8 +151,13 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
   p.lse = lse;
   p.limit_ns = g_wait_limit_ns;
   p.flags = g_flags;
+  p.window = window;
   const unsigned grid = static_cast<unsigned>(p.npairs * s->Hq);
-  if (kv8) {
+  if (window > 0) {
+    static int attrw = set_smem(flash_fwd_kernel<FLASH_SWA, false>, FL_SMEM_DENSE);
+    if (attrw) return attrw;
+    flash_fwd_kernel<FLASH_SWA, false><<<grid, FL_THREADS, FL_SMEM_DENSE, st>>>(mq, mk, mv, p);
+  } else if (kv8) {
     static int attr8 = set_smem(flash_fwd_kernel<FLASH_DENSE, true>, FL_SMEM_KV8);
     if (attr8) return attr8;
     flash_fwd_kernel<FLASH_DENSE, true><<<grid, FL_THREADS, FL_SMEM_KV8, st>>>(mq, mk, mv, p);
@@ -391,6 +397,18 @@ int hs2_attn_fwd(const hs2_shape* shape, const void* q, const void* k, const voi
   if (!q || !o || !lse) return HS2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || !aligned16(lse)) return HS2_ERR_UNSUPPORTED;
   return launch_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, static_cast<cudaStream_t>(stream));
+}
+
+int hs2_swa_attn(const hs2_shape* shape, const void* q, const void* k, const void* v, int32_t window, void* o,
+                 float* lse, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (shape->kv_dtype != HS2_KV_BF16) return HS2_ERR_UNSUPPORTED;
+  if ((rc = check_kv(shape, k, v, nullptr, nullptr))) return rc;
+  if (!q || !o) return HS2_ERR_INVALID_ARG;
+  if (window < 1 || window > shape->L) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || (lse && !aligned16(lse))) return HS2_ERR_UNSUPPORTED;
+  return launch_attn_fwd(shape, q, k, v, nullptr, nullptr, o, lse, static_cast<cudaStream_t>(stream), window);
 }
 
 int hs2_importance(const hs2_shape* shape, const void* q, const void* k, const float* k_scale, const float* lse,

@@ -22,7 +22,7 @@ HS2_KV_BF16, HS2_KV_E4M3 = 0, 1
 EXPORTS = ("hs2_full_attn_select", "hs2_sparse_attn", "hs2_sync", "hs2_attn_fwd", "hs2_importance",
            "hs2_topk_select", "hs2_strerror", "hs2_debug_set", "hs2_version", "hs2_launch_count",
            "hs2_full_attn_select_static", "hs2_exp2_check", "hs2_quantize_kv", "hs2_block_select",
-           "hs2_full_attn_select_blocks")
+           "hs2_full_attn_select_blocks", "hs2_swa_attn")
 
 
 class Hs2Shape(ctypes.Structure):
@@ -51,6 +51,7 @@ _SIGS = {
     "hs2_sparse_attn": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "hs2_sync": [_vp],
     "hs2_attn_fwd": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "hs2_swa_attn": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _i32, _vp, _vp, _vp],
     "hs2_importance": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i64, _vp],
     "hs2_topk_select": [ctypes.POINTER(Hs2Shape), _vp, _i64, _i32, _i32, _vp, _vp, _vp],
     "hs2_debug_set": [_u64, _u32],
@@ -149,6 +150,11 @@ def hs2_sparse_attn(shape, q, k, v, k_scale, v_scale, idx, cnt, o, stream=None) 
 def hs2_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, stream=None) -> None:
     _check(lib().hs2_attn_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale),
                               _ptr(o), _ptr(lse), _stream(stream)), "hs2_attn_fwd")
+
+
+def hs2_swa_attn(shape, q, k, v, window, o, lse=None, stream=None) -> None:
+    _check(lib().hs2_swa_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), int(window), _ptr(o), _ptr(lse),
+                              _stream(stream)), "hs2_swa_attn")
 
 
 def hs2_importance(shape, q, k, k_scale, lse, b0, b1, imp, row_stride, stream=None) -> None:
