@@ -39,7 +39,10 @@ notes of this repository):
   R9  a query row with no visible key (possible only when w < block) gives a
       zero output row;
   R10 FP8 is OCP e4m3fn with one fp32 scale per (token, KV head); a stored
-      value is code * scale.
+      value is code * scale;
+  R13 the sliding window of width W lets query i see keys i - W < j <= i;
+  R14 a decode-step query at position t reuses the list of the block that
+      holds t, with the causal mask j <= t.
 
 Shapes: Q [L][Hq][d], K/V [L][Hkv][d] (token-major), all float64 here.
 """
@@ -328,6 +331,34 @@ def sparse_attn(Q, K, V, idx_row, cnt: int, b: int, g: int, B: int):
         p = np.where(visible, np.exp(s - m), 0.0)
         l = p.sum(axis=1, keepdims=True)
         O[:, hl, :] = np.where(any_vis[:, None], (p @ Vp) / np.where(l > 0, l, 1.0), 0.0)
+    return O
+
+
+def sparse_decode(q_rows, positions, K, V, idx, cnt, B: int):
+    """Decode-step sparse attention ([HS2] KV-sharing paragraph: the sparse
+    layers reuse the full layer's KV cache and token selection; with early
+    exit they mostly run at decode).  Reading R14: a query at position t uses
+    the list of the block holding t, floor(t / B), for its KV head, and sees
+    the listed positions j <= t.
+
+    q_rows [n][Hq][d], positions [n], K / V [L][Hkv][d], idx [Hkv][nb][*],
+    cnt [Hkv][nb].  Returns O [n][Hq][d]; a query with no visible listed key
+    gets a zero row (reading R9)."""
+    n, Hq, d = q_rows.shape
+    G = Hq // K.shape[1]
+    O = np.zeros((n, Hq, d))
+    for r in range(n):
+        t = int(positions[r])
+        b = t // B
+        for h in range(Hq):
+            g = kv_head(h, G)
+            listed = np.asarray(idx[g, b, :int(cnt[g, b])], dtype=np.int64)
+            vis = listed[listed <= t]
+            if vis.size == 0:
+                continue
+            s = (K[vis, g, :] @ q_rows[r, h, :]) / np.sqrt(d)
+            p = np.exp(s - s.max())
+            O[r, h, :] = (p @ V[vis, g, :]) / p.sum()
     return O
 
 

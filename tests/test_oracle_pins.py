@@ -508,3 +508,69 @@ def test_swa_matches_sdpa_with_band_mask():
     Ofull, lfull = orc.swa_attn(Q, K, V, L)         # window >= L is plain causal attention
     Od, ld = orc.dense_attn(Q, K, V)
     assert np.abs(Ofull - Od).max() < 1e-13 and np.abs(lfull - ld).max() < 1e-13
+
+
+# ------------------------------------------------ decode-step sparse attention --
+
+def _full_lists(L, Hkv, B):
+    """Lists holding every position of [0, e_b): the case k >= L."""
+    nb = L // B
+    idx = np.full((Hkv, nb, L), -1, dtype=np.int64)
+    cnt = np.zeros((Hkv, nb), dtype=np.int64)
+    for b in range(nb):
+        e = B * (b + 1)
+        idx[:, b, :e] = np.arange(e)
+        cnt[:, b] = e
+    return idx, cnt
+
+
+def test_decode_with_full_lists_is_causal_attention_rows():
+    L, Hq, Hkv, d, B = 192, 4, 2, 16, 64
+    Q, K, V = _rand((L, Hq, d), 81), _rand((L, Hkv, d), 82), _rand((L, Hkv, d), 83)
+    idx, cnt = _full_lists(L, Hkv, B)
+    pos = np.array([0, 1, 63, 64, 100, 191])
+    O = orc.sparse_decode(Q[pos], pos, K, V, idx, cnt, B)
+    ref = _sdpa(Q, K, V, causal=True)[pos]
+    assert np.abs(O - ref).max() < 1e-12
+
+
+def test_decode_rows_equal_the_block_sparse_layer():
+    """Any query of block b, decoded on its own, gets the row the prefill
+    sparse layer computes for it from the same list."""
+    L, Hq, Hkv, d, B = 256, 8, 2, 16, 64
+    Q, K, V = _rand((L, Hq, d), 84), _rand((L, Hkv, d), 85), _rand((L, Hkv, d), 86)
+    rng = np.random.default_rng(87)
+    nb, width = L // B, 160
+    idx = np.full((Hkv, nb, width), -1, dtype=np.int64)
+    cnt = np.zeros((Hkv, nb), dtype=np.int64)
+    for g in range(Hkv):
+        for b in range(nb):
+            e = B * (b + 1)
+            lst = np.sort(rng.choice(e, size=min(e, width - 40), replace=False))
+            idx[g, b, :lst.size], cnt[g, b] = lst, lst.size
+    G = Hq // Hkv
+    for b in (0, 2, 3):
+        pos = np.arange(B * b, B * (b + 1))
+        O = orc.sparse_decode(Q[pos], pos, K, V, idx, cnt, B)
+        for g in range(Hkv):
+            ref = orc.sparse_attn(Q, K, V, idx[g, b], int(cnt[g, b]), b, g, B)
+            assert np.abs(O[:, g * G:(g + 1) * G] - ref).max() < 1e-12
+
+
+def test_decode_hand_case_and_empty_visibility():
+    """One head, d = 2, a list of three keys: the softmax written out by hand;
+    and a query whose listed keys all lie after it gets a zero row."""
+    K = np.zeros((64, 1, 2))
+    V = np.zeros((64, 1, 2))
+    K[3, 0], K[10, 0], K[40, 0] = [1.0, 0.0], [0.0, 2.0], [3.0, 3.0]
+    V[3, 0], V[10, 0], V[40, 0] = [1.0, 2.0], [-1.0, 0.5], [7.0, 7.0]
+    idx = np.array([[[3, 10, 40, -1]]])
+    cnt = np.array([[3]])
+    q = np.array([[[2.0, 1.0]]])
+    O = orc.sparse_decode(q, np.array([20]), K, V, idx, cnt, 64)   # key 40 is after t = 20
+    s3, s10 = 2.0 / math.sqrt(2), 2.0 / math.sqrt(2)
+    w3, w10 = math.exp(s3), math.exp(s10)
+    want = [(w3 * 1.0 + w10 * -1.0) / (w3 + w10), (w3 * 2.0 + w10 * 0.5) / (w3 + w10)]
+    assert np.abs(O[0, 0] - want).max() < 1e-15
+    O2 = orc.sparse_decode(q, np.array([2]), K, V, idx, cnt, 64)
+    assert np.all(O2 == 0.0)
