@@ -277,6 +277,49 @@ def cpu_baseline(wl, x, seconds_target: float) -> dict:
 
 # ------------------------------------------------------------- cuda arm --
 
+DECODE_BATCHES = (1, 128)   # decode queries per call: one token, and a batch at random positions
+
+
+def decode_rows(hs2, torch, shape, x, k, v, out, dev, timed):
+    """Decode-step sparse attention on the prefill's lists: device time per
+    call and the listed K/V rows the queries must read (plus Q and O)."""
+    res = {}
+    rng = np.random.default_rng(5)
+    peaks = measured_peaks()
+    G = shape.Hq // shape.Hkv
+    for n in DECODE_BATCHES:
+        pos_h = np.array([shape.L - 1] if n == 1 else rng.integers(0, shape.L, n), dtype=np.int64)
+        pos = torch.as_tensor(pos_h, dtype=torch.int32, device=dev)
+        q = x["q_layers"][1][pos.long()].contiguous()
+        sh = hs2.Hs2Shape(**{f: getattr(shape, f) for f, _ in hs2.Hs2Shape._fields_})
+        sh.q_tok_stride, sh.q_head_stride = q.stride(0), q.stride(1)
+        o = torch.empty_like(q)
+        nbytes = hs2.sparse_decode_workspace_bytes(sh, n)
+        ws = torch.empty(nbytes // 4 + 4, dtype=torch.float32, device=dev) if nbytes else None
+        call = lambda: hs2.hs2_sparse_decode(sh, q, pos, k, v, None, None, out["idx"], out["cnt"], o, ws)
+        us_eager = 1e3 * timed(call, 50)
+        # the same calls replayed from a CUDA graph: device time without the
+        # host's per-call cost
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(20):
+                call()
+        us = 1e3 * timed(graph.replay, 5) / 20
+        del graph
+        b = pos.long() // shape.block
+        lists = out["idx"][:, b, :]                       # [Hkv][n][list]
+        cnts = out["cnt"][:, b]                           # [Hkv][n]
+        col = torch.arange(lists.shape[-1], device=dev)
+        vis = (col[None, None, :] < cnts[..., None]) & (lists >= 0) & (lists <= pos[None, :, None])
+        rows = int(vis.sum())
+        moved = rows * 2 * shape.d * k.element_size() + 2 * q.numel() * 2
+        res[f"n{n}"] = {"us_per_call": us, "us_per_call_eager": us_eager, "queries": n, "kv_rows_read": rows, "bytes": moved,
+                        "gbs": moved / (us / 1e6) / 1e9, "frac_of_hbm": moved / (us / 1e6) / 1e9 / peaks["hbm_gbs"],
+                        "splits_workspace_bytes": nbytes}
+        del o, ws
+    return res
+
+
 def run_cuda(args, wl, rank, world, dist):
     import torch
     from token_level_sparse_causal_b200 import build, hs2, inputs
@@ -357,6 +400,7 @@ def run_cuda(args, wl, rank, world, dist):
                    n_stage) if wl.topk % 64 == 0 and k.dtype == torch.bfloat16 else None
     swa_ms = timed(lambda: hs2.hs2_swa_attn(shape, q0, k, v, SWA_WINDOW, out["o"], None, stream),
                    n_stage) if k.dtype == torch.bfloat16 else None
+    decode = decode_rows(hs2, torch, shape, x, k, v, out, dev, timed) if o_sp else None
     hs2.hs2_sync(stream)
 
     # ---- end to end from pinned host buffers through the same C ABI calls
@@ -435,7 +479,8 @@ def run_cuda(args, wl, rank, world, dist):
                                                    work["swa_bytes"] / (peaks["hbm_gbs"] * 1e9)),
                           "frac_of_roofline": 1e3 * max(work["swa_flop"] / (peaks["bf16_tflops"] * 1e12),
                                                         work["swa_bytes"] / (peaks["hbm_gbs"] * 1e9)) / swa_ms,
-                      }},
+                      },
+                      "sparse_decode": decode},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "e2e": e2e,

@@ -203,6 +203,37 @@ int hs2_full_attn_select_blocks(const hs2_shape* shape, const void* q, const voi
                                 const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,
                                 int32_t* cnt, void* workspace, size_t* workspace_bytes, void* stream);
 
+/* ---- decode-step sparse attention ---- */
+
+/*
+ * Sparse-layer attention for n single query tokens at arbitrary positions
+ * (HySparse2 architecture summary, KV-sharing paragraph: the sparse layers
+ * reuse the full layer's KV cache and token selection; with early exit they
+ * mostly run at decode).  Query r at position t = positions[r] attends, for
+ * each KV head g, to the listed positions j <= t of the list of block
+ * floor(t / 64), idx[g][floor(t / 64)][0 .. cnt), with softmax(q.k / sqrt(d)).
+ * A query with no visible listed key gets a zero row.
+ *
+ * shape: the prefill's shape (L, heads, d, topk, recent, kv_dtype, K/V
+ *   strides); its q strides are the strides of `q` and `o` here.
+ * q: bf16 [n][Hq][d]; o: bf16 [n][Hq][d] (written); positions: int32 [n],
+ *   device memory, each in [0, L) (an entry outside it, a count outside
+ *   [0, topk + recent] or a listed position outside [0, e_b) is reported by
+ *   hs2_sync as HS2_ERR_INDEX and never dereferenced; its row is zero).
+ * k, v, k_scale, v_scale, idx, cnt: as hs2_sparse_attn.
+ * workspace: device scratch of hs2_sparse_decode_workspace(shape, n) bytes
+ *   (may be NULL when that is 0), 16-byte aligned; a smaller size returns
+ *   HS2_ERR_WORKSPACE.  It holds no state between calls, but two calls in
+ *   flight at once must not share it.
+ * 1 <= n <= 65535, else HS2_ERR_INVALID_ARG.  Asynchronous on `stream`.
+ */
+int hs2_sparse_decode(const hs2_shape* shape, const void* q, const int32_t* positions, int32_t n, const void* k,
+                      const void* v, const float* k_scale, const float* v_scale, const int32_t* idx,
+                      const int32_t* cnt, void* o, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace size in bytes hs2_sparse_decode needs for (shape, n); host only. */
+int hs2_sparse_decode_workspace(const hs2_shape* shape, int32_t n, size_t* workspace_bytes);
+
 /* ---- sliding-window attention (self-decoder window layers) ---- */
 
 /*

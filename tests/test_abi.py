@@ -178,3 +178,26 @@ def test_swa_argument_checks(lib):
     assert lib.hs2_swa_attn(ctypes.byref(_shape(kv_dtype=1)), P, P, P, 128, P, None, st) == \
         hs2.HS2_ERR_UNSUPPORTED
     assert lib.hs2_swa_attn(ctypes.byref(_shape(d=64)), P, P, P, 128, P, None, st) == hs2.HS2_ERR_UNSUPPORTED
+
+
+def test_decode_workspace_plan_and_argument_checks(lib):
+    st = ctypes.c_void_p(0)
+    s = _shape(L=131072, Hq=64, Hkv=8, q_tok_stride=64 * 128, kv_tok_stride=8 * 128)
+    one = hs2.sparse_decode_workspace_bytes(s, 1)        # 8 units split over 18 chunks
+    assert one >= 8 * 18 * 8 * 128 * 4
+    assert hs2.sparse_decode_workspace_bytes(s, 64) == 0  # 512 units: one CTA each, no partials
+    n = ctypes.c_size_t(0)
+    assert lib.hs2_sparse_decode_workspace(ctypes.byref(s), 0, ctypes.byref(n)) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_sparse_decode_workspace(ctypes.byref(s), 65536, ctypes.byref(n)) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_sparse_decode_workspace(ctypes.byref(s), 1, None) == hs2.HS2_ERR_INVALID_ARG
+    sp = ctypes.byref(s)
+    args = lambda q=P, pos=P, nq=1, o=P, ws=P, wsb=one: (sp, q, pos, nq, P, P, None, None, P, P, o, ws, wsb, st)
+    assert lib.hs2_sparse_decode(*args(ws=P, wsb=one - 4)) == hs2.HS2_ERR_WORKSPACE
+    assert lib.hs2_sparse_decode(*args(ws=None)) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_sparse_decode(*args(q=None)) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_sparse_decode(*args(pos=None)) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_sparse_decode(*args(nq=0)) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_sparse_decode(*args(q=MIS)) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_sparse_decode(*args(ws=MIS)) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_sparse_decode(ctypes.byref(_shape(d=64)), P, P, 1, P, P, None, None, P, P, P, P, one, st) == \
+        hs2.HS2_ERR_UNSUPPORTED

@@ -21,6 +21,7 @@
 #include "importance.cuh"
 #include "topk_select.cuh"
 #include "quantize.cuh"
+#include "decode.cuh"
 
 namespace hs2 {
 namespace {
@@ -211,6 +212,82 @@ int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* 
     static int attr = set_smem(flash_fwd_kernel<FLASH_SPARSE, false>, FL_SMEM_SPARSE);
     if (attr) return attr;
     flash_fwd_kernel<FLASH_SPARSE, false><<<grid, FL_THREADS, FL_SMEM_SPARSE, st>>>(mq, mq, mq, p);
+  }
+  return launched();
+}
+
+// Decode: split each (query, KV head) list so that about three CTAs per SM
+// are in flight even for a single query; a split covers whole 64-entry
+// chunks, and no split is empty for a full list.
+struct DecodePlan {
+  int splits, chunks_per_split;
+  size_t ticket_off, ml_off, part_off, ws_bytes;
+};
+
+DecodePlan decode_plan(const hs2_shape* s, int n) {
+  const int list_len = s->topk + s->recent;
+  const int chunks = (list_len + DEC_CHUNK - 1) / DEC_CHUNK;
+  const int64_t units = static_cast<int64_t>(n) * s->Hkv;
+  const int64_t target = 148 * 3;
+  int splits = static_cast<int>(std::min<int64_t>(chunks, std::max<int64_t>(1, (target + units - 1) / units)));
+  const int cps = (chunks + splits - 1) / splits;
+  splits = (chunks + cps - 1) / cps;
+  DecodePlan pl{splits, cps, 0, 0, 0, 0};
+  if (splits > 1) {
+    const int G = s->Hq / s->Hkv;
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    pl.ticket_off = 0;
+    pl.ml_off = up(static_cast<size_t>(units) * 4);
+    pl.part_off = pl.ml_off + up(static_cast<size_t>(units) * splits * G * 2 * 4);
+    pl.ws_bytes = pl.part_off + static_cast<size_t>(units) * splits * G * 128 * 4;
+  }
+  return pl;
+}
+
+int launch_decode(const hs2_shape* s, const void* q, const int32_t* positions, int n, const void* k, const void* v,
+                  const float* ks, const float* vs, const int32_t* idx, const int32_t* cnt, void* o, void* ws,
+                  const DecodePlan& pl, cudaStream_t st) {
+  DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.q_tok = s->q_tok_stride;
+  p.q_head = s->q_head_stride;
+  p.pos = positions;
+  p.k = static_cast<const uint8_t*>(k);
+  p.v = static_cast<const uint8_t*>(v);
+  p.ksc = ks;
+  p.vsc = vs;
+  p.kv_tok = s->kv_tok_stride;
+  p.kv_head = s->kv_head_stride;
+  p.idx = idx;
+  p.cnt = cnt;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_tok = s->q_tok_stride;
+  p.o_head = s->q_head_stride;
+  p.L = s->L;
+  p.Hkv = s->Hkv;
+  p.G = s->Hq / s->Hkv;
+  p.nb = s->L / 64;
+  p.list_len = s->topk + s->recent;
+  p.block = s->block;
+  p.splits = pl.splits;
+  p.chunks_per_split = pl.chunks_per_split;
+  p.scale_log2 = scale_log2(s->d);
+  if (pl.splits > 1) {
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    p.ticket = reinterpret_cast<unsigned*>(w + pl.ticket_off);
+    p.part_ml = reinterpret_cast<float*>(w + pl.ml_off);
+    p.part_o = reinterpret_cast<float*>(w + pl.part_off);
+    if (int rc = cuda_ok(cudaMemsetAsync(p.ticket, 0, static_cast<size_t>(n) * s->Hkv * 4, st))) return rc;
+  }
+  const dim3 grid(static_cast<unsigned>(pl.splits), static_cast<unsigned>(s->Hkv), static_cast<unsigned>(n));
+  if (s->kv_dtype == HS2_KV_E4M3) {
+    static int attr8 = set_smem(sparse_decode_kernel<true>, DecSmem<true>::BYTES);
+    if (attr8) return attr8;
+    sparse_decode_kernel<true><<<grid, DEC_THREADS, DecSmem<true>::BYTES, st>>>(p);
+  } else {
+    static int attr = set_smem(sparse_decode_kernel<false>, DecSmem<false>::BYTES);
+    if (attr) return attr;
+    sparse_decode_kernel<false><<<grid, DEC_THREADS, DecSmem<false>::BYTES, st>>>(p);
   }
   return launched();
 }
@@ -574,6 +651,30 @@ int hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const 
   if (!q || !o || !idx || !cnt) return HS2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || !aligned16(idx)) return HS2_ERR_UNSUPPORTED;
   return launch_sparse(shape, q, k, v, k_scale, v_scale, idx, cnt, o, static_cast<cudaStream_t>(stream));
+}
+
+int hs2_sparse_decode_workspace(const hs2_shape* shape, int32_t n, size_t* workspace_bytes) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!workspace_bytes || n < 1 || n > 65535) return HS2_ERR_INVALID_ARG;
+  *workspace_bytes = decode_plan(shape, n).ws_bytes;
+  return HS2_OK;
+}
+
+int hs2_sparse_decode(const hs2_shape* shape, const void* q, const int32_t* positions, int32_t n, const void* k,
+                      const void* v, const float* k_scale, const float* v_scale, const int32_t* idx,
+                      const int32_t* cnt, void* o, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (n < 1 || n > 65535) return HS2_ERR_INVALID_ARG;
+  const DecodePlan plan = decode_plan(shape, n);
+  if ((rc = check_kv(shape, k, v, k_scale, v_scale))) return rc;
+  if (!q || !positions || !idx || !cnt || !o) return HS2_ERR_INVALID_ARG;
+  if (plan.ws_bytes > 0 && !workspace) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || (workspace && !aligned16(workspace))) return HS2_ERR_UNSUPPORTED;
+  if (workspace_bytes < plan.ws_bytes) return HS2_ERR_WORKSPACE;
+  return launch_decode(shape, q, positions, n, k, v, k_scale, v_scale, idx, cnt, o, workspace, plan,
+                       static_cast<cudaStream_t>(stream));
 }
 
 int hs2_sync(void* stream) {

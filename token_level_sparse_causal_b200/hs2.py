@@ -22,7 +22,8 @@ HS2_KV_BF16, HS2_KV_E4M3 = 0, 1
 EXPORTS = ("hs2_full_attn_select", "hs2_sparse_attn", "hs2_sync", "hs2_attn_fwd", "hs2_importance",
            "hs2_topk_select", "hs2_strerror", "hs2_debug_set", "hs2_version", "hs2_launch_count",
            "hs2_full_attn_select_static", "hs2_exp2_check", "hs2_quantize_kv", "hs2_block_select",
-           "hs2_full_attn_select_blocks", "hs2_swa_attn")
+           "hs2_full_attn_select_blocks", "hs2_swa_attn", "hs2_sparse_decode",
+           "hs2_sparse_decode_workspace")
 
 
 class Hs2Shape(ctypes.Structure):
@@ -52,6 +53,9 @@ _SIGS = {
     "hs2_sync": [_vp],
     "hs2_attn_fwd": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "hs2_swa_attn": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _i32, _vp, _vp, _vp],
+    "hs2_sparse_decode": [ctypes.POINTER(Hs2Shape), _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                          ctypes.c_size_t, _vp],
+    "hs2_sparse_decode_workspace": [ctypes.POINTER(Hs2Shape), _i32, ctypes.POINTER(ctypes.c_size_t)],
     "hs2_importance": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i64, _vp],
     "hs2_topk_select": [ctypes.POINTER(Hs2Shape), _vp, _i64, _i32, _i32, _vp, _vp, _vp],
     "hs2_debug_set": [_u64, _u32],
@@ -150,6 +154,23 @@ def hs2_sparse_attn(shape, q, k, v, k_scale, v_scale, idx, cnt, o, stream=None) 
 def hs2_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, stream=None) -> None:
     _check(lib().hs2_attn_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale),
                               _ptr(o), _ptr(lse), _stream(stream)), "hs2_attn_fwd")
+
+
+def sparse_decode_workspace_bytes(shape, n: int) -> int:
+    nbytes = ctypes.c_size_t(0)
+    _check(lib().hs2_sparse_decode_workspace(ctypes.byref(shape), int(n), ctypes.byref(nbytes)),
+           "hs2_sparse_decode_workspace")
+    return int(nbytes.value)
+
+
+def hs2_sparse_decode(shape, q, positions, k, v, k_scale, v_scale, idx, cnt, o, workspace=None,
+                      stream=None) -> None:
+    """q / o [n][Hq][d] with the strides in `shape`; positions int32 [n] on the device."""
+    n = int(positions.numel())
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().hs2_sparse_decode(ctypes.byref(shape), _ptr(q), _ptr(positions), n, _ptr(k), _ptr(v),
+                                   _ptr(k_scale), _ptr(v_scale), _ptr(idx), _ptr(cnt), _ptr(o), _ptr(workspace),
+                                   nbytes, _stream(stream)), "hs2_sparse_decode")
 
 
 def hs2_swa_attn(shape, q, k, v, window, o, lse=None, stream=None) -> None:
