@@ -277,6 +277,24 @@ def cpu_baseline(wl, x, seconds_target: float) -> dict:
 
 # ------------------------------------------------------------- cuda arm --
 
+def select_alone(hs2, torch, shape, q0, k, out, dev, timed, nblk=64):
+    """Kernel (3) by itself on the importance rows of the last `nblk` query
+    blocks (the longest rows; a strip larger than L2, so it streams from
+    HBM): device time and the row bytes it must read."""
+    nb = shape.L // shape.block
+    b0 = max(0, nb - nblk)
+    n_c = lambda b: max(0, min(shape.L, shape.block * (b + 1)) - shape.recent)
+    stride = max(4, (n_c(nb - 1) + 3) // 4 * 4)
+    imp = torch.empty((shape.Hkv, nb - b0, stride), dtype=torch.float32, device=dev)
+    hs2.hs2_importance(shape, q0, k, None, out["lse"], b0, nb, imp, stride)
+    ms = timed(lambda: hs2.hs2_topk_select(shape, imp, stride, b0, nb, out["idx"], out["cnt"]), 5)
+    moved = shape.Hkv * 4.0 * sum(n_c(b) for b in range(b0, nb) if n_c(b) > shape.topk)
+    hs2.hs2_sync()
+    del imp
+    return {"blocks": [b0, nb], "ms": ms, "bytes": moved, "gbs": moved / (ms / 1e3) / 1e9,
+            "frac_of_hbm": moved / (ms / 1e3) / 1e9 / measured_peaks()["hbm_gbs"]}
+
+
 DECODE_BATCHES = (1, 128)   # decode queries per call: one token, and a batch at random positions
 
 
@@ -401,6 +419,7 @@ def run_cuda(args, wl, rank, world, dist):
     swa_ms = timed(lambda: hs2.hs2_swa_attn(shape, q0, k, v, SWA_WINDOW, out["o"], None, stream),
                    n_stage) if k.dtype == torch.bfloat16 else None
     decode = decode_rows(hs2, torch, shape, x, k, v, out, dev, timed) if o_sp else None
+    select = select_alone(hs2, torch, shape, q0, k, out, dev, timed)
     hs2.hs2_sync(stream)
 
     # ---- end to end from pinned host buffers through the same C ABI calls
@@ -462,6 +481,7 @@ def run_cuda(args, wl, rank, world, dist):
         "stage_roofline": {
             "fa_fwd_tflops": fa_tflops,
             "importance_select_tflops": work["imp_flop"] / ((fs_ms - fa_ms) / 1e3) / 1e12 if fs_ms > fa_ms else None,
+            "select_alone": select,
             "sparse_tflops": work["sparse_flop"] / (sp_ms / 1e3) / 1e12 if sp_ms else None,
             "sparse_gather_gbs": (work["gather_bytes"] + work["sparse_qo_bytes"]) / (sp_ms / 1e3) / 1e9 if sp_ms else None,
             "path_roofline_ms": 1e3 * ((work["fa_flop"] + work["imp_flop"] + wl.n_sparse * work["sparse_flop"]) /

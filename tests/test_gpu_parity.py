@@ -169,6 +169,43 @@ def test_select_crafted_rows_bit_exact():
         assert np.all(idx_h[:, untouched] == -9) and np.all(cnt_h[:, untouched] == -9)
 
 
+def test_select_rows_that_defeat_the_sample_bit_exact():
+    """Long rows (n > 8192) where the single-read path must give up: all
+    values equal (too many gathered), and a row whose large values sit exactly
+    where a strided sample of 4096 looks, so the sample overestimates the
+    threshold (too few gathered).  The exact radix path then decides, and the
+    lists must still equal the oracle's."""
+    L, Hkv, topk, recent = 16384, 3, 1024, 128
+    shape = hs2.Hs2Shape(L=L, Hq=6, Hkv=Hkv, d=128, block=64, topk=topk, recent=recent, kv_dtype=0,
+                         q_tok_stride=6 * 128, q_head_stride=128, kv_tok_stride=Hkv * 128, kv_head_stride=128)
+    nb = L // 64
+    b0, b1 = nb - 2, nb
+    rng = np.random.default_rng(9)
+    stride = ((orc.n_candidates(64 * b1, recent) + 3) // 4) * 4
+    rows = np.full((Hkv, b1 - b0, stride), np.nan, np.float32)
+    for bi, b in enumerate(range(b0, b1)):
+        n_c = orc.n_candidates(64 * (b + 1), recent)
+        S = 4096
+        sample_pos = (np.arange(S, dtype=np.int64) * n_c) // S + (n_c // S) // 2
+        trap = (rng.random(n_c) * 1e-3).astype(np.float32)
+        trap[sample_pos[:500]] = 1.0          # 500 large values, all of them sampled
+        rows[0, bi, :n_c] = np.full(n_c, 0.25, np.float32)
+        rows[1, bi, :n_c] = trap
+        rows[2, bi, :n_c] = rng.random(n_c).astype(np.float32)
+    imp = torch.from_numpy(rows).to(DEV)
+    idx = torch.full((Hkv, nb, topk + recent), -9, dtype=torch.int32, device=DEV)
+    cnt = torch.full((Hkv, nb), -9, dtype=torch.int32, device=DEV)
+    hs2.hs2_topk_select(shape, imp, stride, b0, b1, idx, cnt)
+    hs2.hs2_sync()
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    for bi, b in enumerate(range(b0, b1)):
+        e_b = 64 * (b + 1)
+        n_c = orc.n_candidates(e_b, recent)
+        for g in range(Hkv):
+            want, wc = orc.select(rows[g, bi, :n_c].astype(np.float64), topk, recent, e_b)
+            assert cnt_h[g, b] == wc and np.array_equal(idx_h[g, b], want), (b, g)
+
+
 # ------------------------------------------------------------ kernel (4) --
 
 def test_sparse_matches_oracle_on_gpu_lists():

@@ -370,7 +370,9 @@ int launch_select(const hs2_shape* s, const float* imp, int64_t row_stride, int 
     if (attr) return attr;
     block_select_kernel<<<grid, SEL_THREADS, dyn, st>>>(p);
   } else {
-    topk_select_kernel<<<grid, SEL_THREADS, 0, st>>>(p);
+    static int attr = set_smem(topk_select_kernel, sizeof(SelSmem));
+    if (attr) return attr;
+    topk_select_kernel<<<grid, SEL_THREADS, sizeof(SelSmem), st>>>(p);
   }
   return launched();
 }
