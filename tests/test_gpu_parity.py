@@ -229,6 +229,51 @@ def test_sparse_matches_oracle_on_gpu_lists():
     assert all(H.guards_intact(bb) for bb in r["bases"])
 
 
+@pytest.mark.parametrize("L,Hq,Hkv", [(3072, 4, 2), (2048, 16, 2), (2560, 8, 1)])
+def test_sparse_group_sizes_match_oracle(L, Hq, Hkv):
+    """G = 2 (one M tile per work item) and G = 8 (two items per block and KV
+    head); every block against the oracle, on GPU lists of 1128 entries (a
+    ragged last key tile)."""
+    wl = _wl(L, Hq, Hkv, n_sparse=1, seed=43, topk=1000)
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    r = H.run_path(wl, xd, guards=True)
+    D = H.decode(x)
+    idx, cnt = r["idx"].cpu().numpy(), r["cnt"].cpu().numpy()
+    G = wl.G
+    got = r["sparse"][0].float().cpu().numpy()
+    ref = np.empty_like(got, dtype=np.float64)
+    for b in range(L // 64):
+        s_b, e_b = orc.block_rows(b, L, 64)
+        for g in range(Hkv):
+            ref[s_b:e_b, g * G:(g + 1) * G] = orc.sparse_attn(D["Q"][1], D["K"], D["V"], idx[g, b], int(cnt[g, b]),
+                                                              b, g, 64)
+    H.bf16_close(got, ref, f"sparse G={G}")
+    assert all(H.guards_intact(bb) for bb in r["bases"])
+
+
+def test_sparse_bounded_wait_reports_timeout_and_context_survives():
+    """The persistent sparse kernel with its load roles switched off (test
+    flag): the MMA and softmax waits run out, hs2_sync reports
+    HS2_ERR_TIMEOUT, and the next call is correct."""
+    wl = _wl(1024, 8, 2, seed=47)
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    r = H.run_path(wl, xd)
+    o = torch.empty_like(xd["q_layers"][1])
+    hs2.hs2_debug_set(50_000_000, 1)
+    try:
+        hs2.hs2_sparse_attn(r["shape"], xd["q_layers"][1], xd["k"], xd["v"], None, None, r["idx"], r["cnt"], o)
+        with pytest.raises(hs2.Hs2Error) as e:
+            hs2.hs2_sync()
+        assert e.value.code == hs2.HS2_ERR_TIMEOUT
+    finally:
+        hs2.hs2_debug_set(H.WAIT_LIMIT_NS, 0)
+    hs2.hs2_sparse_attn(r["shape"], xd["q_layers"][1], xd["k"], xd["v"], None, None, r["idx"], r["cnt"], o)
+    hs2.hs2_sync()
+    assert torch.equal(o, r["sparse"][0])
+
+
 @pytest.mark.parametrize("L", [1152, 640])
 def test_sparse_equals_dense_when_lists_cover_everything(L):
     wl = _wl(L, 8, 2, n_sparse=1, seed=19)

@@ -18,6 +18,7 @@
 #include "../../include/hs2.h"
 #include "common.cuh"
 #include "flash.cuh"
+#include "sparse_attn.cuh"
 #include "importance.cuh"
 #include "topk_select.cuh"
 #include "quantize.cuh"
@@ -107,6 +108,17 @@ int make_map(CUtensorMap* m, const void* base, int L, int H, int64_t tok_stride,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? HS2_OK : HS2_ERR_CUDA;
+}
+
+// Streaming multiprocessors of the current device (queried once per process).
+int sm_count() {
+  static int n = [] {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 148;
+    return v > 0 ? v : 148;
+  }();
+  return n;
 }
 
 float scale_log2(int d) { return static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d))); }
@@ -203,15 +215,17 @@ int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* 
   p.o_head = s->q_head_stride;
   p.limit_ns = g_wait_limit_ns;
   p.flags = g_flags;
-  const unsigned grid = static_cast<unsigned>(p.nb * s->Hkv * p.mpairs);
+  // persistent: one CTA per SM walks the (block, KV head, M-tile pair) items
+  const int n_items = p.nb * s->Hkv * p.mpairs;
+  const unsigned grid = static_cast<unsigned>(std::min(n_items, sm_count()));
   if (s->kv_dtype == HS2_KV_E4M3) {
-    static int attr8 = set_smem(flash_fwd_kernel<FLASH_SPARSE, true>, FL_SMEM_KV8);
+    static int attr8 = set_smem(sparse_attn_kernel<true>, SP_SMEM_KV8);
     if (attr8) return attr8;
-    flash_fwd_kernel<FLASH_SPARSE, true><<<grid, FL_THREADS, FL_SMEM_KV8, st>>>(mq, mq, mq, p);
+    sparse_attn_kernel<true><<<grid, FL_THREADS, SP_SMEM_KV8, st>>>(mq, p, n_items);
   } else {
-    static int attr = set_smem(flash_fwd_kernel<FLASH_SPARSE, false>, FL_SMEM_SPARSE);
+    static int attr = set_smem(sparse_attn_kernel<false>, SP_SMEM);
     if (attr) return attr;
-    flash_fwd_kernel<FLASH_SPARSE, false><<<grid, FL_THREADS, FL_SMEM_SPARSE, st>>>(mq, mq, mq, p);
+    sparse_attn_kernel<false><<<grid, FL_THREADS, SP_SMEM, st>>>(mq, p, n_items);
   }
   return launched();
 }

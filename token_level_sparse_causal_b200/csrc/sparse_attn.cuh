@@ -1,0 +1,604 @@
+// Kernel (4), persistent: the sparse layers' attention over the shared index
+// lists (HySparse2 architecture summary, KV-sharing paragraph: the sparse
+// layers reuse the full layer's KV cache and token selection), with the
+// causal mask j <= i on listed positions.
+//
+// The arithmetic per work item is that of flash_fwd_kernel<FLASH_SPARSE>: an
+// item is (query block b, KV head g, pair of 128-row M tiles), each M tile
+// 128/G tokens x G heads of the block sharing the block's list, whose K/V rows
+// are gathered with 16-byte cp.async into 128-byte-swizzled shared memory
+// and multiplied on tcgen05 tensor cores (S in TMEM, P written back over S,
+// O += P V from TMEM).  An item touches only 1152 keys (9 key tiles), so a
+// CTA per item spends as long on its start and end -- TMEM allocation,
+// barrier set-up, the Q and list loads, the first gathers, the last softmax
+// and the O write -- as on the tiles themselves.  Here one CTA per SM loops
+// over items instead, and every pipeline keeps running across item
+// boundaries:
+//
+//   * the K/V ring, the per-tile barriers and TMEM carry over: phases are
+//     counted over the CTA's whole tile stream, not per item;
+//   * Q of the next item is loaded as soon as the last S of the current one
+//     has executed (q_empty), while its last P V products and softmax run;
+//   * the index list is double-buffered (list_full / list_empty), so the
+//     gather of the next item starts while the current one is finishing;
+//   * the first P V of an item waits only for the previous epilogue of the
+//     same M tile to have read O (o_free); its S products do not wait.
+//
+// Roles (12 warps), as in flash_fwd_kernel: warp 0 loads Q by TMA, warp 1
+// issues every MMA, warps 2-3 load lists and gather K/V (with an FP8 cache:
+// also convert Q and the K/V codes to f16), warps 4-7 / 8-11 run the softmax
+// and epilogue of M tile A / B.  Every wait is bounded; a wait that runs out
+// records HS2_ERR_TIMEOUT and the CTA winds down.
+#pragma once
+
+#include "flash.cuh"
+
+namespace hs2 {
+
+struct SparseBars {
+  uint64_t q_raw;    // KV8: Q landed (bf16), before its conversion
+  uint64_t q_full;   // Q of the current item ready for the MMAs
+  uint64_t q_empty;  // the item's last S products have executed
+  uint64_t full_k[FL_STAGES];
+  uint64_t full_v[FL_STAGES];
+  uint64_t empty[FL_STAGES];  // a stage's K/V rows: both P V products of its tile have executed
+  uint64_t s_full[2];
+  uint64_t p_ready[2];
+  uint64_t o_done[2];
+  uint64_t o_free[2];  // epilogue of M tile x has read O
+  uint64_t list_full[2];
+  uint64_t list_empty[2];
+  uint64_t fin;
+  uint32_t tmem_slot;
+  int abort;
+};
+static_assert(sizeof(SparseBars) <= 256, "barriers fit their slot");
+
+constexpr uint32_t SP_POS_OFF = FL_POS_OFF;                      // int [2][MAX_LIST]
+constexpr uint32_t SP_KSC_OFF = SP_POS_OFF + 2 * MAX_LIST * 4;   // KV8: [stage][128]
+constexpr uint32_t SP_SMEM = SP_KSC_OFF + 1024;                  // + alignment slack
+constexpr uint32_t SP_SMEM_KV8 = SP_KSC_OFF + FL_STAGES * 128 * 4 + 1024;
+
+struct SpItem {
+  int b, g, pair, cnt, nt, nB, e_b;
+  bool has_b;
+};
+
+// The list length of item `it` (0 past the last item).
+__device__ __forceinline__ int item_cnt(const FlashParams& p, int it, int n_items) {
+  if (it >= n_items) return 0;
+  const int bg = it / p.mpairs;
+  return __ldg(p.cnt + static_cast<int64_t>(bg % p.Hkv) * p.nb + bg / p.Hkv);
+}
+
+// Item `it` given its list length c (read one item ahead, off the critical path).
+__device__ __forceinline__ SpItem sparse_item(const FlashParams& p, int it, int c) {
+  SpItem w;
+  w.pair = it % p.mpairs;
+  const int bg = it / p.mpairs;
+  w.g = bg % p.Hkv;
+  w.b = bg / p.Hkv;
+  w.e_b = min(p.L, 64 * (w.b + 1));
+  w.cnt = max(0, min(c, p.list_len));
+  w.nt = (w.cnt + 127) / 128;
+  w.has_b = 2 * w.pair + 1 < p.mtiles;
+  w.nB = w.has_b ? w.nt : 0;
+  return w;
+}
+
+template <bool KV8>
+__global__ void __launch_bounds__(FL_THREADS, 1)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const FlashParams p, int n_items) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  SparseBars* bars = reinterpret_cast<SparseBars*>(smem + FL_BAR_OFF);
+  int32_t* pos_base = reinterpret_cast<int32_t*>(smem + SP_POS_OFF);
+  float* ksc_s = reinterpret_cast<float*>(smem + SP_KSC_OFF);
+  const uint32_t q_base = smem_u32(smem + FL_Q_OFF);
+  const uint32_t kv_base = smem_u32(smem + FL_KV_OFF);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &bars->abort;
+  const int first = blockIdx.x, step = gridDim.x;
+  // loader threads: warps 2-3 with an FP8 cache (warp 0 then only loads Q);
+  // warps 0, 2, 3 with bf16, warp 0's lane 0 also loading Q
+  constexpr int NLD = KV8 ? 64 : 96;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_raw, 1);
+    mbar_init(&bars->q_full, KV8 ? 64u : 1u);
+    mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < FL_STAGES; ++s) {
+      mbar_init(&bars->full_k[s], NLD);
+      mbar_init(&bars->full_v[s], NLD);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->p_ready[x], 128);
+      mbar_init(&bars->o_done[x], 1);
+      mbar_init(&bars->o_free[x], 128);
+      mbar_init(&bars->list_full[x], NLD);
+      mbar_init(&bars->list_empty[x], 256);
+    }
+    mbar_init(&bars->fin, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_slot;
+
+  if (KV8 && warp == 0) {
+    // ========================================================= Q by TMA
+    if (lane == 0 && !(p.flags & FLAG_SKIP_LOADS)) {
+      tma_prefetch_desc(&tmQ);
+      uint64_t* qbar = KV8 ? &bars->q_raw : &bars->q_full;
+      int ii = 0, loaded = 0;
+      int c_cur = item_cnt(p, first, n_items), c_nxt = 0;
+      for (int it = first; it < n_items; it += step, ++ii, c_cur = c_nxt) {
+        c_nxt = item_cnt(p, it + step, n_items);
+        const SpItem w = sparse_item(p, it, c_cur);
+        if (w.nt == 0) continue;
+        if (loaded > 0 && !mbar_wait(&bars->q_empty, (loaded - 1) & 1, p.limit_ns, abort_flag, 301)) break;
+        const int nq = w.has_b ? 2 : 1;
+        mbar_arrive_expect_tx(qbar, static_cast<uint32_t>(nq) * TILE_BYTES);
+        for (int x = 0; x < nq; ++x) {
+          uint8_t* qd = smem + FL_Q_OFF + x * TILE_BYTES;
+          const int t0 = 64 * w.b + (2 * w.pair + x) * p.rows_tok;
+          tma_load_3d(qd, &tmQ, qbar, 0, w.g * p.G, t0);
+          tma_load_3d(qd + HALF_BYTES, &tmQ, qbar, 64, w.g * p.G, t0);
+        }
+        ++loaded;
+      }
+      // never leave a TMA write in flight into memory the CTA gives back
+      if (loaded > 0) wait_done(qbar, (loaded - 1) & 1, p.limit_ns, 302);
+    }
+  } else if (warp == 1) {
+    // ========================================================== MMA issue
+    if (lane == 0) {
+      int u0 = 0, qi = 0;            // tiles of the CTA's stream so far; items with Q
+      int tx[2] = {0, 0}, jx[2] = {0, 0};  // tiles / items per M tile so far
+      bool ok = true;
+      int c_cur = item_cnt(p, first, n_items), c_nxt = 0;
+      for (int it = first; it < n_items && ok; it += step, c_cur = c_nxt) {
+        c_nxt = item_cnt(p, it + step, n_items);
+        const SpItem w = sparse_item(p, it, c_cur);
+        const int nt = w.nt;
+        if (nt == 0) continue;
+        const int nx[2] = {nt, w.nB};
+        auto issue_s = [&](int x, int j) {
+          const uint32_t kb = kv_base + ((u0 + j) % FL_STAGES) * 2 * TILE_BYTES;
+          const uint32_t qb = q_base + x * TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+            umma_ss(tmem + x * 128, sdesc_sw128(qb + koff, 16, 1024), sdesc_sw128(kb + koff, 16, 1024),
+                    KV8 ? IDESC_S_F16 : IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars->s_full[x]);
+        };
+        auto issue_pv = [&](int x, int j) {
+          const uint32_t vb = kv_base + ((u0 + j) % FL_STAGES) * 2 * TILE_BYTES + TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t bdesc = sdesc_sw128(vb + kk * 2048, HALF_BYTES, 1024);
+            umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bdesc, KV8 ? IDESC_PV_F16 : IDESC_PV,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars->o_done[x]);
+        };
+        ok = mbar_wait(&bars->q_full, qi & 1, p.limit_ns, abort_flag, 311);
+        if (ok) ok = mbar_wait(&bars->full_k[u0 % FL_STAGES], (u0 / FL_STAGES) & 1, p.limit_ns, abort_flag, 312);
+        if (!ok) break;
+        tc_fence_after();
+        for (int x = 0; x < 2; ++x)
+          if (nx[x] > 0) issue_s(x, 0);
+        if (nt == 1) umma_commit(&bars->q_empty);
+        for (int j = 0; j < nt && ok; ++j) {
+          const int u = u0 + j;
+          const int s = u % FL_STAGES;
+          bool v_ready = false, k_next = false;
+          for (int x = 0; x < 2 && ok; ++x) {
+            if (j >= nx[x]) continue;
+            if (!mbar_wait(&bars->p_ready[x], (tx[x] + j) & 1, p.limit_ns, abort_flag, 313)) {
+              ok = false;
+              break;
+            }
+            if (!v_ready) {
+              if (!mbar_wait(&bars->full_v[s], (u / FL_STAGES) & 1, p.limit_ns, abort_flag, 314)) {
+                ok = false;
+                break;
+              }
+              v_ready = true;
+            }
+            // the first P V of an item overwrites O: the previous epilogue must have read it
+            if (j == 0 && jx[x] > 0 &&
+                !mbar_wait(&bars->o_free[x], (jx[x] - 1) & 1, p.limit_ns, abort_flag, 315)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(x, j);
+            // the tile's last P V is issued: its stage is released as soon as
+            // that executes, before the next tile's S products are queued
+            if (x == 1 || j >= nx[1]) umma_commit(&bars->empty[s]);
+            if (j + 1 < nx[x]) {
+              if (!k_next) {
+                const int s1 = (u + 1) % FL_STAGES;
+                if (!mbar_wait(&bars->full_k[s1], ((u + 1) / FL_STAGES) & 1, p.limit_ns, abort_flag, 316)) {
+                  ok = false;
+                  break;
+                }
+                k_next = true;
+                tc_fence_after();
+              }
+              issue_s(x, j + 1);
+            }
+          }
+          if (ok && j + 2 == nt) umma_commit(&bars->q_empty);  // the item's last S products are issued
+        }
+        u0 += nt;
+        ++qi;
+        for (int x = 0; x < 2; ++x) {
+          tx[x] += nx[x];
+          jx[x] += nx[x] > 0 ? 1 : 0;
+        }
+      }
+      umma_commit(&bars->fin);
+      wait_done(&bars->fin, 0, p.limit_ns, 317);
+    }
+  } else if (warp == 0 || warp == 2 || warp == 3) {
+    // ===================================== lists and K/V (gather / convert)
+    if (!(p.flags & FLAG_SKIP_LOADS)) {
+      const int pt = KV8 ? threadIdx.x - 64 : (warp == 0 ? lane : threadIdx.x - 32);  // 0 .. NLD-1
+      const bool q_thread = !KV8 && warp == 0 && lane == 0;
+      if (q_thread) tma_prefetch_desc(&tmQ);
+      int ii = 0, u0 = 0, qi = 0, loaded = 0;
+      bool ok = true;
+      int c_cur = item_cnt(p, first, n_items), c_nxt = 0;
+      for (int it = first; it < n_items && ok; it += step, ++ii, c_cur = c_nxt) {
+        c_nxt = item_cnt(p, it + step, n_items);
+        const SpItem w = sparse_item(p, it, c_cur);
+        const int buf = ii & 1;
+        int32_t* pos_s = pos_base + buf * MAX_LIST;
+        // ---- the item's list (the buffer's previous item is done with it)
+        if (ii >= 2 && !mbar_wait(&bars->list_empty[buf], ((ii >> 1) - 1) & 1, p.limit_ns, abort_flag, 321)) {
+          ok = false;
+          break;
+        }
+        if (q_thread && w.nt > 0) {  // bf16: Q of the item, once the previous item's S products ran
+          if (loaded > 0 && !mbar_wait(&bars->q_empty, (loaded - 1) & 1, p.limit_ns, abort_flag, 301)) {
+            ok = false;
+            break;
+          }
+          const int nq = w.has_b ? 2 : 1;
+          mbar_arrive_expect_tx(&bars->q_full, static_cast<uint32_t>(nq) * TILE_BYTES);
+          for (int x = 0; x < nq; ++x) {
+            uint8_t* qd = smem + FL_Q_OFF + x * TILE_BYTES;
+            const int t0 = 64 * w.b + (2 * w.pair + x) * p.rows_tok;
+            tma_load_3d(qd, &tmQ, &bars->q_full, 0, w.g * p.G, t0);
+            tma_load_3d(qd + HALF_BYTES, &tmQ, &bars->q_full, 64, w.g * p.G, t0);
+          }
+          ++loaded;
+        }
+        // entries past the count, and entries outside [0, e_b) (reported),
+        // become -1: never read, always masked
+        const int32_t* list = p.idx + (static_cast<int64_t>(w.g) * p.nb + w.b) * p.list_len;
+        for (int i = pt; i < w.nt * 128; i += NLD) {
+          int e = -1;
+          if (i < w.cnt) {
+            e = __ldg(list + i);
+            if (e < 0 || e >= w.e_b) {
+              report(HS2_ERR_INDEX, 328);
+              e = -1;
+            }
+          }
+          pos_s[i] = e;
+        }
+        mbar_arrive(&bars->list_full[buf]);
+        // the loaders read each other's entries too: wait for all of them (bounded)
+        if (!mbar_wait(&bars->list_full[buf], (ii >> 1) & 1, p.limit_ns, abort_flag, 327)) {
+          ok = false;
+          break;
+        }
+        if (w.nt == 0) continue;
+        if (KV8) {
+          // ---- Q: bf16 -> f16 in place, once its TMA has landed
+          if (!mbar_wait(&bars->q_raw, qi & 1, p.limit_ns, abort_flag, 322)) {
+            ok = false;
+            break;
+          }
+          const int nchunks = (w.has_b ? 2 : 1) * static_cast<int>(TILE_BYTES / 16);
+          for (int c = pt; c < nchunks; c += 64) {
+            const uint32_t a = q_base + c * 16;
+            st_shared_v4(a, bf16x8_to_f16x8(ld_shared_v4(a)));
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&bars->q_full);
+          // ---- K/V tiles: 8 threads per 128-byte code row
+          const int rsub = pt >> 3, c8 = pt & 7;
+          const uint8_t* kb8 = p.k8 + static_cast<int64_t>(w.g) * p.kv_head + c8 * 16;
+          const uint8_t* vb8 = p.v8 + static_cast<int64_t>(w.g) * p.kv_head + c8 * 16;
+          for (int j = 0; j < w.nt && ok; ++j) {
+            const int u = u0 + j;
+            const int s = u % FL_STAGES;
+            if (u >= FL_STAGES &&
+                !mbar_wait(&bars->empty[s], ((u / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 323)) {
+              ok = false;
+              break;
+            }
+            const uint32_t kd = kv_base + s * 2 * TILE_BYTES;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {  // 0: K, 1: V
+              const uint8_t* base8 = half ? vb8 : kb8;
+              const float* scale = half ? p.vsc : p.ksc;
+#pragma unroll 4
+              for (int i = 0; i < 16; ++i) {
+                const int r = rsub + 8 * i;
+                const int gi = j * 128 + r;
+                const int pj = pos_s[gi];
+                const bool valid = pj >= 0;
+                uint4 raw = make_uint4(0, 0, 0, 0);
+                float sg = 0.f;
+                if (valid) {
+                  raw = ld_nc_v4(base8 + static_cast<int64_t>(pj) * p.kv_tok);
+                  sg = scale[static_cast<int64_t>(pj) * p.Hkv + w.g];
+                }
+                const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+                uint32_t f[8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  f[2 * q] = e4m3x2_to_f16x2(wd[q]);
+                  f[2 * q + 1] = e4m3x2_to_f16x2(wd[q] >> 16);
+                }
+                if (half) {
+                  const uint32_t s2 = pack_f16x2(sg, sg);
+#pragma unroll
+                  for (int q = 0; q < 8; ++q) f[q] = hmul2_u32(f[q], s2);
+                } else if (c8 == 0) {
+                  ksc_s[s * 128 + r] = sg * p.scale_log2;
+                }
+                const uint32_t dst = kd + half * TILE_BYTES;
+                st_shared_v4(dst + sw128_chunk_offset(r, 2 * c8, 128), make_uint4(f[0], f[1], f[2], f[3]));
+                st_shared_v4(dst + sw128_chunk_offset(r, 2 * c8 + 1, 128), make_uint4(f[4], f[5], f[6], f[7]));
+              }
+              fence_proxy_async_smem();
+              mbar_arrive(half ? &bars->full_v[s] : &bars->full_k[s]);
+            }
+          }
+        } else {
+          // ---- bf16 gather: per key tile, 16 threads per row (one 16-byte
+          // chunk each) and 6 rows at a time, K and V of a row together
+          const int rg = pt >> 4, chunk = pt & 15;
+          const uint32_t half_off = static_cast<uint32_t>((chunk >> 3) * 128 * 128);
+          const __nv_bfloat16* kg = p.k + static_cast<int64_t>(w.g) * p.kv_head + chunk * 8;
+          const __nv_bfloat16* vg = p.v + static_cast<int64_t>(w.g) * p.kv_head + chunk * 8;
+          for (int j = 0; j < w.nt && ok; ++j) {
+            const int u = u0 + j;
+            const int s = u % FL_STAGES;
+            if (u >= FL_STAGES &&
+                !mbar_wait(&bars->empty[s], ((u / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 325)) {
+              ok = false;
+              break;
+            }
+            const uint32_t kd = kv_base + s * 2 * TILE_BYTES + half_off;
+            const int32_t* pj_row = pos_s + j * 128;
+#pragma unroll 6
+            for (int r = rg; r < 128; r += NLD / 16) {
+              const int pj = pj_row[r];
+              const bool valid = pj >= 0;
+              const int64_t off = static_cast<int64_t>(valid ? pj : 0) * p.kv_tok;
+              const uint32_t d = kd + static_cast<uint32_t>(r * 128 + (((chunk & 7) ^ (r & 7)) << 4));
+              cp_async_16(d, kg + off, valid ? 16u : 0u);
+              cp_async_16(d + TILE_BYTES, vg + off, valid ? 16u : 0u);
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->full_k[s]);
+            mbar_arrive(&bars->full_v[s]);
+          }
+        }
+        u0 += w.nt;
+        ++qi;
+      }
+      cp_async_wait<0>();
+      if (q_thread && loaded > 0) wait_done(&bars->q_full, (loaded - 1) & 1, p.limit_ns, 302);
+    }
+  } else {
+    // ============================================ softmax / rescale / epilogue
+    const int x = (warp >= 8) ? 1 : 0;  // M tile of this warpgroup
+    const int r = threadIdx.x - 128 - 128 * x;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_tm = tmem + lane_off + x * 128;
+    const uint32_t o_tm = tmem + lane_off + 256 + x * 128;
+    const float sc = KV8 ? 1.f : p.scale_log2;  // KV8 folds the scale into the columns
+    int ii = 0, u0 = 0, tx = 0;
+    bool ok = true;
+    int c_cur = item_cnt(p, first, n_items), c_nxt = 0;
+    for (int it = first; it < n_items && ok; it += step, ++ii, c_cur = c_nxt) {
+      c_nxt = item_cnt(p, it + step, n_items);
+      const SpItem w = sparse_item(p, it, c_cur);
+      const int buf = ii & 1;
+      const int32_t* pos_s = pos_base + buf * MAX_LIST;
+      const int nX = x ? w.nB : w.nt;
+      const int mt = 2 * w.pair + x;
+      const int i_row = 64 * w.b + mt * p.rows_tok + r / p.G;
+      const int hh = w.g * p.G + r % p.G;
+      const int i_min = 64 * w.b + mt * p.rows_tok;
+      if (!warp_wait(&bars->list_full[buf], (ii >> 1) & 1, p.limit_ns, abort_flag, 330)) {
+        ok = false;
+        break;
+      }
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < nX; ++j) {
+        const int t = tx + j;  // tiles this M tile has seen before j
+        if (!warp_wait(&bars->s_full[x], t & 1, p.limit_ns, abort_flag, 331)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sr[4][32];
+        tmem_ld32(s_tm, sr[0]);
+        tmem_ld32(s_tm + 32, sr[1]);
+        tmem_ld32(s_tm + 64, sr[2]);
+        tmem_ld32(s_tm + 96, sr[3]);
+        tmem_ld_wait();
+        reg_fence(sr[0]);
+        reg_fence(sr[1]);
+        reg_fence(sr[2]);
+        reg_fence(sr[3]);
+        if (KV8) {  // per-key scale (already times log2(e)/sqrt(d)) on every column
+          const uint64_t* ks2 = reinterpret_cast<const uint64_t*>(ksc_s + ((u0 + j) % FL_STAGES) * 128);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float a0, a1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])),
+                               ks2[c * 16 + e]),
+                        a0, a1);
+              sr[c][2 * e] = __float_as_uint(a0);
+              sr[c][2 * e + 1] = __float_as_uint(a1);
+            }
+          }
+        }
+        // ---- causal mask on listed positions (after any scaling)
+        const int last = j * 128 + 127;
+        if ((last >= w.cnt) || (pos_s[last] > i_min)) {
+          const int4* pv4 = reinterpret_cast<const int4*>(pos_s + j * 128);
+#pragma unroll
+          for (int c4 = 0; c4 < 32; ++c4) {
+            const int4 q4 = pv4[c4];  // same address in every lane: a broadcast
+            const int pj[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = c4 * 4 + e;
+              const bool keep = (j * 128 + c < w.cnt) && (pj[e] >= 0) && (pj[e] <= i_row);
+              if (!keep) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+            }
+          }
+        }
+        // ---- row max: 4 independent chains of 3-input max
+        float mx4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) mx4[q] = __uint_as_float(sr[q][0]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int e = 0; e < 15; ++e)
+            mx4[q] = fmax3(mx4[q], __uint_as_float(sr[q][1 + 2 * e]), __uint_as_float(sr[q][2 + 2 * e]));
+          mx4[q] = fmaxf(mx4[q], __uint_as_float(sr[q][31]));
+        }
+        const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
+        const float m_new = fmaxf(m_used, mx * sc);
+        float alpha = 1.f;
+        const bool resc = m_new > m_used + 8.f;
+        if (resc) {
+          alpha = ex2_approx(m_used - m_new);
+          m_used = m_new;
+        }
+        const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+        l *= alpha;
+        // ---- P = exp2(s * scale - m) into TMEM over S
+        const uint64_t sc2 = f2_pack(sc, sc), nmu2 = f2_pack(-mu, -mu);
+        uint64_t sum2[2] = {0ull, 0ull};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t a2 =
+                f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])), sc2, nmu2);
+            const uint64_t p2 = ex2_x2(a2);
+            sum2[e & 1] = f2_add(sum2[e & 1], p2);
+            float e0, e1;
+            f2_unpack(p2, e0, e1);
+            pk[e] = KV8 ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
+          }
+          tmem_st16(s_tm + c * 16, pk);
+        }
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(sum2[0], a0, a1);
+          f2_unpack(sum2[1], b0, b1);
+          l += (a0 + a1) + (b0 + b1);
+        }
+        // ---- O rescale (needs P V of the previous tile complete)
+        if (j > 0) {
+          if (!warp_wait(&bars->o_done[x], (t - 1) & 1, p.limit_ns, abort_flag, 332)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t orr[32];
+              tmem_ld32(o_tm + c * 32, orr);
+              tmem_ld_wait();
+              reg_fence(orr);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+              tmem_st32(o_tm + c * 32, orr);
+            }
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->p_ready[x]);
+      }
+      mbar_arrive(&bars->list_empty[buf]);  // masking is done with this list
+      if (!ok) break;
+      // ---- epilogue
+      const bool row_live = x == 0 || w.has_b;
+      __nv_bfloat16* orow = p.o + static_cast<int64_t>(i_row) * p.o_tok + static_cast<int64_t>(hh) * p.o_head;
+      if (nX > 0) {
+        if (!warp_wait(&bars->o_done[x], (tx + nX - 1) & 1, p.limit_ns, abort_flag, 333)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(o_tm + c * 32, orr);
+          tmem_ld_wait();
+          reg_fence(orr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->o_free[x]);
+      } else if (w.nt == 0 && row_live) {
+        // an empty list: the rows attend to nothing
+        uint4* dst = reinterpret_cast<uint4*>(orow);
+        for (int v4 = 0; v4 < 16; ++v4) dst[v4] = make_uint4(0, 0, 0, 0);
+      }
+      u0 += w.nt;
+      tx += nX;
+    }
+  }
+
+  // ---- teardown: every role has drained its asynchronous work
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace hs2
