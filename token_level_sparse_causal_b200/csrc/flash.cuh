@@ -1,5 +1,6 @@
 // Flash-attention forward on tcgen05 tensor cores, in two modes sharing one
-// pipeline:
+// pipeline (the sparse layers' kernel in sparse_attn.cuh is built on the same
+// pipeline):
 //
 //   FLASH_DENSE  -- kernel (1): causal grouped-query attention of the full
 //                   layer, one CTA per (pair of 128-query tiles, query head),
@@ -8,13 +9,6 @@
 //                   summary, ablation paragraph: the full layer's complete
 //                   scores; SHARP walk-through, section 1.1:
 //                   softmax(Q K^T / sqrt(d)) V.)
-//   FLASH_SPARSE -- kernel (4): a sparse layer (KV Reuse, KV-sharing
-//                   paragraph), one CTA per (query block b, KV head g, pair of
-//                   128-row M tiles); each M tile is (128/G tokens) x (G heads)
-//                   of the block, all sharing the block's index list, whose K/V
-//                   rows are gathered with 16-byte cp.async into swizzled
-//                   shared memory; the causal mask j <= i applies to listed
-//                   positions.
 //   FLASH_SWA    -- causal sliding-window attention of the self-decoder's
 //                   window layers (HySparse2 architecture summary, paragraph
 //                   on the self-decoder / cross-decoder split): the dense
@@ -23,10 +17,10 @@
 //                   i - window < j <= i.  bf16 cache only.
 //
 // CTA = 12 warps:
-//   warp 0      TMA: Q tiles (both modes), K/V tiles (dense)
+//   warp 0      TMA: Q tiles, K/V tiles (bf16 cache)
 //   warp 1      TMEM allocation; one thread issues every tcgen05.mma
-//   warps 2-3   K/V gather (sparse, bf16 cache); with an FP8 cache: convert Q
-//               to f16 in place, then load, convert and scale every K/V tile
+//   warps 2-3   with an FP8 cache: convert Q to f16 in place, then load,
+//               convert and scale every K/V tile
 //   warps 4-7   softmax / rescale / epilogue of query tile A (thread r <-> row r)
 //   warps 8-11  the same for query tile B
 //
@@ -68,7 +62,6 @@ constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
 constexpr uint32_t IDESC_S_F16 = idesc_f16_f32(128, 128, 0, 0);
 constexpr uint32_t IDESC_PV_F16 = idesc_f16_f32(128, 128, 0, 1);
 constexpr int FLASH_DENSE = 0;
-constexpr int FLASH_SPARSE = 1;
 constexpr int FLASH_SWA = 2;
 constexpr uint32_t FLAG_SKIP_LOADS = 1u;
 constexpr int MAX_LIST = 4096;
@@ -114,7 +107,6 @@ constexpr uint32_t FL_KV_OFF = 2 * TILE_BYTES;  // stage s: K at +0, V at +TILE_
 constexpr uint32_t FL_BAR_OFF = FL_KV_OFF + FL_STAGES * 2 * TILE_BYTES;
 constexpr uint32_t FL_POS_OFF = FL_BAR_OFF + 256;
 constexpr uint32_t FL_SMEM_DENSE = FL_POS_OFF + 1024;  // + alignment slack
-constexpr uint32_t FL_SMEM_SPARSE = FL_POS_OFF + MAX_LIST * 4 + 1024;
 constexpr uint32_t FL_KSC_OFF = FL_POS_OFF + MAX_LIST * 4;  // KV8: [stage][128] column scales
 constexpr uint32_t FL_SMEM_KV8 = FL_KSC_OFF + FL_STAGES * 128 * 4 + 1024;
 
@@ -149,7 +141,6 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   FlashBars* bars = reinterpret_cast<FlashBars*>(smem + FL_BAR_OFF);
-  int32_t* pos_s = reinterpret_cast<int32_t*>(smem + FL_POS_OFF);
   float* ksc_s = reinterpret_cast<float*>(smem + FL_KSC_OFF);
   const uint32_t q_base = smem_u32(smem + FL_Q_OFF);
   const uint32_t kv_base = smem_u32(smem + FL_KV_OFF);
@@ -158,45 +149,28 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
 
   // ---- work item: query tiles A and B (B may be absent); query tile x uses
   // key tiles lo(x) .. (x ? nB : nA) - 1 (lo is 0 except in SWA mode)
-  constexpr bool kDenseLike = MODE != FLASH_SPARSE;
-  int h = 0, g = 0, b = 0, pair = 0, cnt = 0, e_b = 0, nA = 0, nB = 0;
+  // KV-group-major order, longest tile pairs first within a group: the CTAs
+  // resident at any time share one group's K/V, which then stays in L2.
+  const int per_g = p.npairs * p.G;
+  const int g = static_cast<int>(blockIdx.x) / per_g;
+  const int rem = static_cast<int>(blockIdx.x) % per_g;
+  const int pair = p.npairs - 1 - rem / p.G;
+  const int h = g * p.G + rem % p.G;
+  const int nA = 2 * pair + 1;
+  const int nB = (2 * pair + 1 < p.nqt) ? 2 * pair + 2 : 0;
   int lo0 = 0, lo1 = 0;  // first key tile of query tile A / B
-  if (kDenseLike) {
-    // KV-group-major order, longest tile pairs first within a group: the
-    // CTAs resident at any time share one group's K/V, which then stays in L2.
-    const int per_g = p.npairs * p.G;
-    g = static_cast<int>(blockIdx.x) / per_g;
-    const int rem = static_cast<int>(blockIdx.x) % per_g;
-    pair = p.npairs - 1 - rem / p.G;
-    h = g * p.G + rem % p.G;
-    nA = 2 * pair + 1;
-    nB = (2 * pair + 1 < p.nqt) ? 2 * pair + 2 : 0;
-    if (MODE == FLASH_SWA) {
-      lo0 = max(0, 2 * pair * 128 - p.window + 1) / 128;
-      lo1 = max(0, (2 * pair + 1) * 128 - p.window + 1) / 128;
-    }
-  } else {
-    pair = static_cast<int>(blockIdx.x) % p.mpairs;
-    const int bg = static_cast<int>(blockIdx.x) / p.mpairs;
-    g = bg % p.Hkv;
-    b = bg / p.Hkv;
-    e_b = min(p.L, 64 * (b + 1));
-    cnt = p.cnt[static_cast<int64_t>(g) * p.nb + b];
-    cnt = max(0, min(cnt, p.list_len));
-    const int nt = (cnt + 127) / 128;
-    nA = nt;
-    nB = (2 * pair + 1 < p.mtiles) ? nt : 0;
-    const int32_t* list = p.idx + (static_cast<int64_t>(g) * p.nb + b) * p.list_len;
-    for (int i = threadIdx.x; i < nt * 128; i += blockDim.x) pos_s[i] = (i < cnt) ? list[i] : -1;
+  if (MODE == FLASH_SWA) {
+    lo0 = max(0, 2 * pair * 128 - p.window + 1) / 128;
+    lo1 = max(0, (2 * pair + 1) * 128 - p.window + 1) / 128;
   }
   const int n = max(nA, nB);
   const int j0 = lo0;  // first key tile of the CTA (lo0 <= lo1)
   // a compile-time 0 outside SWA mode
   auto lo = [&](int x) { return MODE == FLASH_SWA ? (x ? lo1 : lo0) : 0; };
-  const bool has_b = kDenseLike ? (nB > 0) : (2 * pair + 1 < p.mtiles);
+  const bool has_b = nB > 0;
 
   if (threadIdx.x == 0) {
-    const uint32_t kv_arrivals = (kDenseLike && !KV8) ? 1u : 64u;
+    const uint32_t kv_arrivals = KV8 ? 64u : 1u;
     mbar_init(&bars->q_raw, 1);
     mbar_init(&bars->q_full, KV8 ? 64u : 1u);
     for (int s = 0; s < FL_STAGES; ++s) {
@@ -231,16 +205,10 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       mbar_arrive_expect_tx(qbar, static_cast<uint32_t>(nq) * TILE_BYTES);
       for (int x = 0; x < nq; ++x) {
         uint8_t* qd = smem + FL_Q_OFF + x * TILE_BYTES;
-        if (kDenseLike) {
-          tma_load_3d(qd, &tmQ, qbar, 0, h, (2 * pair + x) * 128);
-          tma_load_3d(qd + HALF_BYTES, &tmQ, qbar, 64, h, (2 * pair + x) * 128);
-        } else {
-          const int t0 = 64 * b + (2 * pair + x) * p.rows_tok;
-          tma_load_3d(qd, &tmQ, qbar, 0, g * p.G, t0);
-          tma_load_3d(qd + HALF_BYTES, &tmQ, qbar, 64, g * p.G, t0);
-        }
+        tma_load_3d(qd, &tmQ, qbar, 0, h, (2 * pair + x) * 128);
+        tma_load_3d(qd + HALF_BYTES, &tmQ, qbar, 64, h, (2 * pair + x) * 128);
       }
-      if (kDenseLike && !KV8) {
+      if (!KV8) {
         int last = -1;
         for (int j = j0; j < n; ++j) {
           const int u = j - j0;  // position in this CTA's key-tile stream
@@ -379,18 +347,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
 #pragma unroll 4
             for (int it = 0; it < 16; ++it) {
               const int r = rsub + 8 * it;
-              int pj;
-              bool valid;
-              if (MODE == FLASH_DENSE) {
-                pj = j * 128 + r;
-                valid = pj < p.L;
-              } else {
-                const int gi = j * 128 + r;
-                pj = pos_s[gi];
-                const bool listed = gi < cnt;
-                valid = listed && pj >= 0 && pj < e_b;
-                if (!half && listed && !valid) report(HS2_ERR_INDEX, 143);
-              }
+              const int pj = j * 128 + r;
+              const bool valid = pj < p.L;
               uint4 raw = make_uint4(0, 0, 0, 0);
               float sg = 0.f;
               if (valid) {
@@ -420,52 +378,6 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           }
         }
       }
-    } else if (MODE == FLASH_SPARSE && !KV8 && !(p.flags & FLAG_SKIP_LOADS)) {
-      // ========================================================= K/V gather
-      const int pt = threadIdx.x - 64;  // 0..63
-      const int row_sub = (pt >> 4) & 1, chunk = pt & 15, pw = pt >> 5;
-      const __nv_bfloat16* kg = p.k + static_cast<int64_t>(g) * p.kv_head + chunk * 8;
-      const __nv_bfloat16* vg = p.v + static_cast<int64_t>(g) * p.kv_head + chunk * 8;
-      // Per key tile: K rows then V rows as two cp.async groups; K is
-      // published as soon as it lands so S can start while V is in flight.
-      // A tile is published before the next stage is awaited: the MMA order
-      // needs tile j+1's K before it can release tile j's stage.
-      for (int j = 0; j < n; ++j) {
-        const int s = j % FL_STAGES;
-        if (j >= FL_STAGES &&
-            !mbar_wait(&bars->empty[s], ((j / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 121))
-          break;
-        const uint32_t kd = kv_base + s * 2 * TILE_BYTES;
-#pragma unroll 4
-        for (int it = 0; it < 32; ++it) {
-          const int r = pw * 2 + row_sub + 4 * it;
-          const int gi = j * 128 + r;
-          const int pj = pos_s[gi];
-          const bool listed = gi < cnt;
-          const bool valid = listed && pj >= 0 && pj < e_b;
-          if (listed && !valid) report(HS2_ERR_INDEX, 122);
-          const int64_t off = static_cast<int64_t>(valid ? pj : 0) * p.kv_tok;
-          cp_async_16(kd + sw128_chunk_offset(r, chunk, 128), kg + off, valid ? 16u : 0u);
-        }
-        cp_async_commit();
-#pragma unroll 4
-        for (int it = 0; it < 32; ++it) {
-          const int r = pw * 2 + row_sub + 4 * it;
-          const int gi = j * 128 + r;
-          const int pj = pos_s[gi];
-          const bool valid = gi < cnt && pj >= 0 && pj < e_b;
-          const int64_t off = static_cast<int64_t>(valid ? pj : 0) * p.kv_tok;
-          cp_async_16(kd + TILE_BYTES + sw128_chunk_offset(r, chunk, 128), vg + off, valid ? 16u : 0u);
-        }
-        cp_async_commit();
-        cp_async_wait<1>();
-        fence_proxy_async_smem();
-        mbar_arrive(&bars->full_k[s]);
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(&bars->full_v[s]);
-      }
-      cp_async_wait<0>();
     }
   } else {
     // ============================================ softmax / rescale / epilogue
@@ -475,19 +387,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t s_tm = tmem + lane_off + x * 128;
     const uint32_t o_tm = tmem + lane_off + 256 + x * 128;
-    int i_row, hh, i_min, diag = -1;
-    if (kDenseLike) {
-      const int qt = 2 * pair + x;
-      i_row = qt * 128 + r;
-      hh = h;
-      i_min = qt * 128;
-      diag = qt;
-    } else {
-      const int mt = 2 * pair + x;
-      i_row = 64 * b + mt * p.rows_tok + r / p.G;
-      hh = g * p.G + r % p.G;
-      i_min = 64 * b + mt * p.rows_tok;
-    }
+    const int qt = 2 * pair + x;
+    const int i_row = qt * 128 + r, hh = h, i_min = qt * 128, diag = qt;
     const float sc = KV8 ? 1.f : p.scale_log2;  // KV8 folds the scale into the columns
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -527,35 +428,19 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       bool need_mask;
       if (MODE == FLASH_DENSE) {
         need_mask = (j == diag);
-      } else if (MODE == FLASH_SWA) {  // the diagonal, or keys below some row's window
+      } else {  // the diagonal, or keys below some row's window
         need_mask = (j == diag) || (j * 128 < i_min + 128 - p.window);
-      } else {
-        const int last = j * 128 + 127;
-        need_mask = (last >= cnt) || (pos_s[last] > i_min);
       }
       if (need_mask) {
         if (MODE == FLASH_DENSE) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c > r) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-        } else if (MODE == FLASH_SWA) {  // keep i - window < j*128 + c <= i
+        } else {  // keep i - window < j*128 + c <= i
           const int c_hi = i_row - j * 128, c_lo = c_hi - p.window;
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c > c_hi || c <= c_lo) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-        } else {
-          const int4* pv4 = reinterpret_cast<const int4*>(pos_s + j * 128);
-#pragma unroll
-          for (int c4 = 0; c4 < 32; ++c4) {
-            const int4 q4 = pv4[c4];  // same address in every lane: a broadcast
-            const int pj[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = c4 * 4 + e;
-              const bool keep = (j * 128 + c < cnt) && (pj[e] >= 0) && (pj[e] <= i_row);
-              if (!keep) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-            }
-          }
         }
       }
       // ---- row max: 4 independent chains of 3-input max
@@ -652,12 +537,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
             dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
       }
-      if (kDenseLike && row_live && (MODE == FLASH_DENSE || p.lse != nullptr))
+      if (row_live && (MODE == FLASH_DENSE || p.lse != nullptr))
         p.lse[static_cast<int64_t>(hh) * p.L + i_row] = (m_used + log2f(l)) * 0.69314718055994530942f;
-    } else if (MODE == FLASH_SPARSE && ok && n == 0 && row_live) {
-      // an empty list: the rows attend to nothing
-      uint4* dst = reinterpret_cast<uint4*>(orow);
-      for (int v4 = 0; v4 < 16; ++v4) dst[v4] = make_uint4(0, 0, 0, 0);
     }
   }
 
