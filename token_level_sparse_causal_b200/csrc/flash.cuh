@@ -1,6 +1,6 @@
-// Flash-attention forward on tcgen05 tensor cores, in two modes sharing one
-// pipeline (the sparse layers' kernel in sparse_attn.cuh is built on the same
-// pipeline):
+// Flash-attention forward on tcgen05 tensor cores (the sparse layers' and
+// the sliding window's persistent kernel in sparse_attn.cuh is built on the
+// same pipeline):
 //
 //   FLASH_DENSE  -- kernel (1): causal grouped-query attention of the full
 //                   layer, one CTA per (pair of 128-query tiles, query head),
@@ -9,12 +9,6 @@
 //                   summary, ablation paragraph: the full layer's complete
 //                   scores; SHARP walk-through, section 1.1:
 //                   softmax(Q K^T / sqrt(d)) V.)
-//   FLASH_SWA    -- causal sliding-window attention of the self-decoder's
-//                   window layers (HySparse2 architecture summary, paragraph
-//                   on the self-decoder / cross-decoder split): the dense
-//                   pipeline with query tile x starting at key tile lo(x),
-//                   the first one that meets the window, and a band mask
-//                   i - window < j <= i.  bf16 cache only.
 //
 // CTA = 12 warps:
 //   warp 0      TMA: Q tiles, K/V tiles (bf16 cache)
@@ -62,7 +56,6 @@ constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
 constexpr uint32_t IDESC_S_F16 = idesc_f16_f32(128, 128, 0, 0);
 constexpr uint32_t IDESC_PV_F16 = idesc_f16_f32(128, 128, 0, 1);
 constexpr int FLASH_DENSE = 0;
-constexpr int FLASH_SWA = 2;
 constexpr uint32_t FLAG_SKIP_LOADS = 1u;
 constexpr int MAX_LIST = 4096;
 
@@ -71,7 +64,7 @@ struct FlashParams {
   int nb, list_len, mtiles, rows_tok;  // sparse: blocks, list stride, M tiles per (b,g), tokens per M tile
   int mpairs;                          // sparse: pairs of M tiles per (b,g)
   float scale_log2;                    // log2(e) / sqrt(d)
-  int window;                          // SWA: keys i - window < j <= i
+  int window;                          // window mode of the persistent kernel: keys i - window < j <= i
   const __nv_bfloat16* k;              // gather sources (sparse)
   const __nv_bfloat16* v;
   const uint8_t* k8;                   // e4m3 codes and fp32 scales [L][Hkv] (KV8)
@@ -137,7 +130,7 @@ template <int MODE, bool KV8>
 __global__ void __launch_bounds__(FL_THREADS, 1)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const FlashParams p) {
-  static_assert(!(MODE == FLASH_SWA && KV8), "the window mode reads a bf16 cache");
+  static_assert(MODE == FLASH_DENSE, "one mode: causal attention + LSE");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   FlashBars* bars = reinterpret_cast<FlashBars*>(smem + FL_BAR_OFF);
@@ -148,7 +141,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
   volatile int* abort_flag = &bars->abort;
 
   // ---- work item: query tiles A and B (B may be absent); query tile x uses
-  // key tiles lo(x) .. (x ? nB : nA) - 1 (lo is 0 except in SWA mode)
+  // key tiles 0 .. (x ? nB : nA) - 1
   // KV-group-major order, longest tile pairs first within a group: the CTAs
   // resident at any time share one group's K/V, which then stays in L2.
   const int per_g = p.npairs * p.G;
@@ -158,15 +151,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
   const int h = g * p.G + rem % p.G;
   const int nA = 2 * pair + 1;
   const int nB = (2 * pair + 1 < p.nqt) ? 2 * pair + 2 : 0;
-  int lo0 = 0, lo1 = 0;  // first key tile of query tile A / B
-  if (MODE == FLASH_SWA) {
-    lo0 = max(0, 2 * pair * 128 - p.window + 1) / 128;
-    lo1 = max(0, (2 * pair + 1) * 128 - p.window + 1) / 128;
-  }
   const int n = max(nA, nB);
-  const int j0 = lo0;  // first key tile of the CTA (lo0 <= lo1)
-  // a compile-time 0 outside SWA mode
-  auto lo = [&](int x) { return MODE == FLASH_SWA ? (x ? lo1 : lo0) : 0; };
+
   const bool has_b = nB > 0;
 
   if (threadIdx.x == 0) {
@@ -210,8 +196,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       }
       if (!KV8) {
         int last = -1;
-        for (int j = j0; j < n; ++j) {
-          const int u = j - j0;  // position in this CTA's key-tile stream
+        for (int j = 0; j < n; ++j) {
+          const int u = j;  // position in this CTA's key-tile stream
           const int s = u % FL_STAGES;
           if (u >= FL_STAGES &&
               !mbar_wait(&bars->empty[s], ((u / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 101))
@@ -239,7 +225,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     if (lane == 0 && n > 0) {
       const int nx[2] = {nA, nB};
       auto issue_s = [&](int x, int j) {
-        const uint32_t kb = kv_base + ((j - j0) % FL_STAGES) * 2 * TILE_BYTES;
+        const uint32_t kb = kv_base + (j % FL_STAGES) * 2 * TILE_BYTES;
         const uint32_t qb = q_base + x * TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -250,12 +236,12 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         umma_commit(&bars->s_full[x]);
       };
       auto issue_pv = [&](int x, int j) {
-        const uint32_t vb = kv_base + ((j - j0) % FL_STAGES) * 2 * TILE_BYTES + TILE_BYTES;
+        const uint32_t vb = kv_base + (j % FL_STAGES) * 2 * TILE_BYTES + TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bdesc = sdesc_sw128(vb + kk * 2048, HALF_BYTES, 1024);
           umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bdesc, KV8 ? IDESC_PV_F16 : IDESC_PV,
-                  (j > lo(x) || kk > 0) ? 1u : 0u);
+                  (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars->o_done[x]);
       };
@@ -264,15 +250,15 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       if (ok) {
         tc_fence_after();
         for (int x = 0; x < 2; ++x)
-          if (nx[x] > lo(x) && lo(x) == j0) issue_s(x, j0);
+          if (nx[x] > 0) issue_s(x, 0);
       }
-      for (int j = j0; j < n && ok; ++j) {
-        const int u = j - j0;
+      for (int j = 0; j < n && ok; ++j) {
+        const int u = j;
         const int s = u % FL_STAGES;
         bool v_ready = false, k_next = false;
         for (int x = 0; x < 2 && ok; ++x) {
-          if (j < lo(x) || j >= nx[x]) continue;
-          if (!mbar_wait(&bars->p_ready[x], (j - lo(x)) & 1, p.limit_ns, abort_flag, 113)) {
+          if (j >= nx[x]) continue;
+          if (!mbar_wait(&bars->p_ready[x], j & 1, p.limit_ns, abort_flag, 113)) {
             ok = false;
             break;
           }
@@ -289,21 +275,6 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
             if (!k_next) {
               const int s1 = (u + 1) % FL_STAGES;
               if (!mbar_wait(&bars->full_k[s1], ((u + 1) / FL_STAGES) & 1, p.limit_ns, abort_flag, 115)) {
-                ok = false;
-                break;
-              }
-              k_next = true;
-              tc_fence_after();
-            }
-            issue_s(x, j + 1);
-          }
-        }
-        // a query tile whose first key tile is the next one starts now
-        for (int x = 0; x < 2 && ok && MODE == FLASH_SWA; ++x) {
-          if (lo(x) == j + 1 && j + 1 < nx[x]) {
-            if (!k_next) {
-              const int s1 = (u + 1) % FL_STAGES;
-              if (!mbar_wait(&bars->full_k[s1], ((u + 1) / FL_STAGES) & 1, p.limit_ns, abort_flag, 116)) {
                 ok = false;
                 break;
               }
@@ -388,12 +359,12 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     const uint32_t s_tm = tmem + lane_off + x * 128;
     const uint32_t o_tm = tmem + lane_off + 256 + x * 128;
     const int qt = 2 * pair + x;
-    const int i_row = qt * 128 + r, hh = h, i_min = qt * 128, diag = qt;
+    const int i_row = qt * 128 + r, hh = h, diag = qt;
     const float sc = KV8 ? 1.f : p.scale_log2;  // KV8 folds the scale into the columns
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = lo(x); j < nX; ++j) {
-      const int t = j - lo(x);  // tiles this query tile has seen before j
+    for (int j = 0; j < nX; ++j) {
+      const int t = j;  // tiles this query tile has seen before j
       if (!warp_wait(&bars->s_full[x], t & 1, p.limit_ns, abort_flag, 131)) {
         ok = false;
         break;
@@ -425,23 +396,10 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         }
       }
       // ---- mask (after any scaling, so a masked column is exactly -inf)
-      bool need_mask;
-      if (MODE == FLASH_DENSE) {
-        need_mask = (j == diag);
-      } else {  // the diagonal, or keys below some row's window
-        need_mask = (j == diag) || (j * 128 < i_min + 128 - p.window);
-      }
-      if (need_mask) {
-        if (MODE == FLASH_DENSE) {
+      if (j == diag) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c > r) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-        } else {  // keep i - window < j*128 + c <= i
-          const int c_hi = i_row - j * 128, c_lo = c_hi - p.window;
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c > c_hi || c <= c_lo) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-        }
+        for (int c = 0; c < 128; ++c)
+          if (c > r) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
       }
       // ---- row max: 4 independent chains of 3-input max
       float mx4[4];
@@ -516,7 +474,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     // ---- epilogue
     const bool row_live = i_row < p.L && (x == 0 || has_b);  // a last dense tile may hang past L
     __nv_bfloat16* orow = p.o + static_cast<int64_t>(i_row) * p.o_tok + static_cast<int64_t>(hh) * p.o_head;
-    const int nT = nX - lo(x);  // key tiles of this query tile
+    const int nT = nX;  // key tiles of this query tile
     if (ok && nT > 0 && warp_wait(&bars->o_done[x], (nT - 1) & 1, p.limit_ns, abort_flag, 133)) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
@@ -537,7 +495,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
             dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
       }
-      if (row_live && (MODE == FLASH_DENSE || p.lse != nullptr))
+      if (row_live)
         p.lse[static_cast<int64_t>(hh) * p.L + i_row] = (m_used + log2f(l)) * 0.69314718055994530942f;
     }
   }

@@ -130,9 +130,8 @@ int set_smem(K kernel, uint32_t bytes) {
 
 // ------------------------------------------------------------- launches --
 
-// window > 0 launches the sliding-window mode (bf16 cache only).
 int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void* v, const float* ks,
-                    const float* vs, void* o, float* lse, cudaStream_t st, int window = 0) {
+                    const float* vs, void* o, float* lse, cudaStream_t st) {
   const bool kv8 = s->kv_dtype == HS2_KV_E4M3;
   CUtensorMap mq, mk, mv;
   int rc;
@@ -164,13 +163,8 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
   p.lse = lse;
   p.limit_ns = g_wait_limit_ns;
   p.flags = g_flags;
-  p.window = window;
   const unsigned grid = static_cast<unsigned>(p.npairs * s->Hq);
-  if (window > 0) {
-    static int attrw = set_smem(flash_fwd_kernel<FLASH_SWA, false>, FL_SMEM_DENSE);
-    if (attrw) return attrw;
-    flash_fwd_kernel<FLASH_SWA, false><<<grid, FL_THREADS, FL_SMEM_DENSE, st>>>(mq, mk, mv, p);
-  } else if (kv8) {
+  if (kv8) {
     static int attr8 = set_smem(flash_fwd_kernel<FLASH_DENSE, true>, FL_SMEM_KV8);
     if (attr8) return attr8;
     flash_fwd_kernel<FLASH_DENSE, true><<<grid, FL_THREADS, FL_SMEM_KV8, st>>>(mq, mk, mv, p);
@@ -182,13 +176,22 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
   return launched();
 }
 
+// The persistent kernel (4): over index lists, or (window > 0) over each
+// block's sliding windows, bf16 cache, optionally writing the LSE.
 int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* v, const float* ks,
-                  const float* vs, const int32_t* idx, const int32_t* cnt, void* o, cudaStream_t st) {
+                  const float* vs, const int32_t* idx, const int32_t* cnt, void* o, cudaStream_t st, int window = 0,
+                  float* lse = nullptr) {
   const int G = s->Hq / s->Hkv;
   const int rows_tok = 128 / G;
-  CUtensorMap mq;
+  CUtensorMap mq, mk, mv;
   int rc;
   if ((rc = make_map(&mq, q, s->L, s->Hq, s->q_tok_stride, s->q_head_stride, G, rows_tok))) return rc;
+  mk = mq;
+  mv = mq;
+  if (window > 0) {
+    if ((rc = make_map(&mk, k, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+    if ((rc = make_map(&mv, v, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+  }
   FlashParams p{};
   p.L = s->L;
   p.Hq = s->Hq;
@@ -200,6 +203,7 @@ int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* 
   p.mpairs = (p.mtiles + 1) / 2;
   p.rows_tok = rows_tok;
   p.scale_log2 = scale_log2(s->d);
+  p.window = window;
   p.k = static_cast<const __nv_bfloat16*>(k);
   p.v = static_cast<const __nv_bfloat16*>(v);
   p.k8 = static_cast<const uint8_t*>(k);
@@ -213,19 +217,24 @@ int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* 
   p.o = static_cast<__nv_bfloat16*>(o);
   p.o_tok = s->q_tok_stride;
   p.o_head = s->q_head_stride;
+  p.lse = lse;
   p.limit_ns = g_wait_limit_ns;
   p.flags = g_flags;
   // persistent: one CTA per SM walks the (block, KV head, M-tile pair) items
   const int n_items = p.nb * s->Hkv * p.mpairs;
   const unsigned grid = static_cast<unsigned>(std::min(n_items, sm_count()));
-  if (s->kv_dtype == HS2_KV_E4M3) {
-    static int attr8 = set_smem(sparse_attn_kernel<true>, SP_SMEM_KV8);
+  if (window > 0) {
+    static int attrw = set_smem(sparse_attn_kernel<false, true>, SP_SMEM);
+    if (attrw) return attrw;
+    sparse_attn_kernel<false, true><<<grid, FL_THREADS, SP_SMEM, st>>>(mq, mk, mv, p, n_items);
+  } else if (s->kv_dtype == HS2_KV_E4M3) {
+    static int attr8 = set_smem(sparse_attn_kernel<true, false>, SP_SMEM_KV8);
     if (attr8) return attr8;
-    sparse_attn_kernel<true><<<grid, FL_THREADS, SP_SMEM_KV8, st>>>(mq, p, n_items);
+    sparse_attn_kernel<true, false><<<grid, FL_THREADS, SP_SMEM_KV8, st>>>(mq, mk, mv, p, n_items);
   } else {
-    static int attr = set_smem(sparse_attn_kernel<false>, SP_SMEM);
+    static int attr = set_smem(sparse_attn_kernel<false, false>, SP_SMEM);
     if (attr) return attr;
-    sparse_attn_kernel<false><<<grid, FL_THREADS, SP_SMEM, st>>>(mq, p, n_items);
+    sparse_attn_kernel<false, false><<<grid, FL_THREADS, SP_SMEM, st>>>(mq, mk, mv, p, n_items);
   }
   return launched();
 }
@@ -501,7 +510,8 @@ int hs2_swa_attn(const hs2_shape* shape, const void* q, const void* k, const voi
   if (!q || !o) return HS2_ERR_INVALID_ARG;
   if (window < 1 || window > shape->L) return HS2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || (lse && !aligned16(lse))) return HS2_ERR_UNSUPPORTED;
-  return launch_attn_fwd(shape, q, k, v, nullptr, nullptr, o, lse, static_cast<cudaStream_t>(stream), window);
+  return launch_sparse(shape, q, k, v, nullptr, nullptr, nullptr, nullptr, o, static_cast<cudaStream_t>(stream),
+                       window, lse);
 }
 
 int hs2_importance(const hs2_shape* shape, const void* q, const void* k, const float* k_scale, const float* lse,

@@ -1,7 +1,12 @@
 // Kernel (4), persistent: the sparse layers' attention over the shared index
 // lists (HySparse2 architecture summary, KV-sharing paragraph: the sparse
 // layers reuse the full layer's KV cache and token selection), with the
-// causal mask j <= i on listed positions.
+// causal mask j <= i on listed positions.  Window mode (WIN): the same
+// pipeline computes causal sliding-window attention (the self-decoder's window
+// layers; HySparse2 architecture summary, paragraph on the self-decoder /
+// cross-decoder split): an item's keys are the contiguous range its block's
+// windows cover, loaded as whole tiles by TMA, with the band mask
+// i - W < j <= i.
 //
 // The arithmetic per work item is that of flash_fwd_kernel<FLASH_SPARSE>: an
 // item is (query block b, KV head g, pair of 128-row M tiles), each M tile
@@ -61,6 +66,7 @@ constexpr uint32_t SP_SMEM_KV8 = SP_KSC_OFF + FL_STAGES * 128 * 4 + 1024;
 
 struct SpItem {
   int b, g, pair, cnt, nt, nB, e_b;
+  int lo;  // window mode: the first key of the item's contiguous key range
   bool has_b;
 };
 
@@ -71,7 +77,10 @@ __device__ __forceinline__ int item_cnt(const FlashParams& p, int it, int n_item
   return __ldg(p.cnt + static_cast<int64_t>(bg % p.Hkv) * p.nb + bg / p.Hkv);
 }
 
-// Item `it` given its list length c (read one item ahead, off the critical path).
+// Item `it` given its list length c (read one item ahead, off the critical
+// path).  In window mode the keys are the contiguous range the block's
+// windows cover, [max(0, 64 b - W + 1), 64 b + 63], and c is not used.
+template <bool WIN>
 __device__ __forceinline__ SpItem sparse_item(const FlashParams& p, int it, int c) {
   SpItem w;
   w.pair = it % p.mpairs;
@@ -79,16 +88,23 @@ __device__ __forceinline__ SpItem sparse_item(const FlashParams& p, int it, int 
   w.g = bg % p.Hkv;
   w.b = bg / p.Hkv;
   w.e_b = min(p.L, 64 * (w.b + 1));
-  w.cnt = max(0, min(c, p.list_len));
+  w.lo = 0;
+  if (WIN) {
+    w.lo = max(0, 64 * w.b - p.window + 1);
+    c = w.e_b - w.lo;
+  }
+  w.cnt = max(0, min(c, WIN ? c : p.list_len));
   w.nt = (w.cnt + 127) / 128;
   w.has_b = 2 * w.pair + 1 < p.mtiles;
   w.nB = w.has_b ? w.nt : 0;
   return w;
 }
 
-template <bool KV8>
+template <bool KV8, bool WIN>
 __global__ void __launch_bounds__(FL_THREADS, 1)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const FlashParams p, int n_items) {
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const FlashParams p, int n_items) {
+  static_assert(!(KV8 && WIN), "the window mode reads a bf16 cache");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   SparseBars* bars = reinterpret_cast<SparseBars*>(smem + FL_BAR_OFF);
@@ -108,8 +124,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     mbar_init(&bars->q_full, KV8 ? 64u : 1u);
     mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < FL_STAGES; ++s) {
-      mbar_init(&bars->full_k[s], NLD);
-      mbar_init(&bars->full_v[s], NLD);
+      mbar_init(&bars->full_k[s], WIN ? 1 : NLD);
+      mbar_init(&bars->full_v[s], WIN ? 1 : NLD);
       mbar_init(&bars->empty[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
@@ -133,17 +149,41 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_slot;
 
-  if (KV8 && warp == 0) {
-    // ========================================================= Q by TMA
+  if ((KV8 || WIN) && warp == 0) {
+    // ============================ Q by TMA (and, in window mode, K/V tiles)
     if (lane == 0 && !(p.flags & FLAG_SKIP_LOADS)) {
       tma_prefetch_desc(&tmQ);
+      if (WIN) {
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+      }
+      int u0 = 0, last_u = -1;
       uint64_t* qbar = KV8 ? &bars->q_raw : &bars->q_full;
       int ii = 0, loaded = 0;
-      int c_cur = item_cnt(p, first, n_items), c_nxt = 0;
+      int c_cur = WIN ? 0 : item_cnt(p, first, n_items), c_nxt = 0;
       for (int it = first; it < n_items; it += step, ++ii, c_cur = c_nxt) {
-        c_nxt = item_cnt(p, it + step, n_items);
-        const SpItem w = sparse_item(p, it, c_cur);
+        c_nxt = WIN ? 0 : item_cnt(p, it + step, n_items);
+        const SpItem w = sparse_item<WIN>(p, it, c_cur);
         if (w.nt == 0) continue;
+        bool ok = true;
+        // window mode: key tile j of the item into its ring stage
+        auto load_tile = [&](int j) -> bool {
+          const int u = u0 + j;
+          const int s = u % FL_STAGES;
+          if (u >= FL_STAGES &&
+              !mbar_wait(&bars->empty[s], ((u / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 305))
+            return false;
+          uint8_t* kd = smem + FL_KV_OFF + s * 2 * TILE_BYTES;
+          const int t0 = w.lo + j * 128;
+          mbar_arrive_expect_tx(&bars->full_k[s], TILE_BYTES);
+          tma_load_3d(kd, &tmK, &bars->full_k[s], 0, w.g, t0);
+          tma_load_3d(kd + HALF_BYTES, &tmK, &bars->full_k[s], 64, w.g, t0);
+          mbar_arrive_expect_tx(&bars->full_v[s], TILE_BYTES);
+          tma_load_3d(kd + TILE_BYTES, &tmV, &bars->full_v[s], 0, w.g, t0);
+          tma_load_3d(kd + TILE_BYTES + HALF_BYTES, &tmV, &bars->full_v[s], 64, w.g, t0);
+          last_u = u;
+          return true;
+        };
         if (loaded > 0 && !mbar_wait(&bars->q_empty, (loaded - 1) & 1, p.limit_ns, abort_flag, 301)) break;
         const int nq = w.has_b ? 2 : 1;
         mbar_arrive_expect_tx(qbar, static_cast<uint32_t>(nq) * TILE_BYTES);
@@ -154,9 +194,16 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           tma_load_3d(qd + HALF_BYTES, &tmQ, qbar, 64, w.g * p.G, t0);
         }
         ++loaded;
+        for (int j = 0; WIN && j < w.nt && ok; ++j) ok = load_tile(j);
+        if (!ok) break;
+        u0 += w.nt;
       }
       // never leave a TMA write in flight into memory the CTA gives back
       if (loaded > 0) wait_done(qbar, (loaded - 1) & 1, p.limit_ns, 302);
+      for (int u = max(0, last_u - FL_STAGES + 1); u <= last_u; ++u) {
+        wait_done(&bars->full_k[u % FL_STAGES], (u / FL_STAGES) & 1, p.limit_ns, 306);
+        wait_done(&bars->full_v[u % FL_STAGES], (u / FL_STAGES) & 1, p.limit_ns, 307);
+      }
     }
   } else if (warp == 1) {
     // ========================================================== MMA issue
@@ -164,10 +211,10 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       int u0 = 0, qi = 0;            // tiles of the CTA's stream so far; items with Q
       int tx[2] = {0, 0}, jx[2] = {0, 0};  // tiles / items per M tile so far
       bool ok = true;
-      int c_cur = item_cnt(p, first, n_items), c_nxt = 0;
+      int c_cur = WIN ? 0 : item_cnt(p, first, n_items), c_nxt = 0;
       for (int it = first; it < n_items && ok; it += step, c_cur = c_nxt) {
-        c_nxt = item_cnt(p, it + step, n_items);
-        const SpItem w = sparse_item(p, it, c_cur);
+        c_nxt = WIN ? 0 : item_cnt(p, it + step, n_items);
+        const SpItem w = sparse_item<WIN>(p, it, c_cur);
         const int nt = w.nt;
         if (nt == 0) continue;
         const int nx[2] = {nt, w.nB};
@@ -252,7 +299,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       umma_commit(&bars->fin);
       wait_done(&bars->fin, 0, p.limit_ns, 317);
     }
-  } else if (warp == 0 || warp == 2 || warp == 3) {
+  } else if (!WIN && (warp == 0 || warp == 2 || warp == 3)) {
     // ===================================== lists and K/V (gather / convert)
     if (!(p.flags & FLAG_SKIP_LOADS)) {
       const int pt = KV8 ? threadIdx.x - 64 : (warp == 0 ? lane : threadIdx.x - 32);  // 0 .. NLD-1
@@ -260,10 +307,10 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       if (q_thread) tma_prefetch_desc(&tmQ);
       int ii = 0, u0 = 0, qi = 0, loaded = 0;
       bool ok = true;
-      int c_cur = item_cnt(p, first, n_items), c_nxt = 0;
+      int c_cur = WIN ? 0 : item_cnt(p, first, n_items), c_nxt = 0;
       for (int it = first; it < n_items && ok; it += step, ++ii, c_cur = c_nxt) {
-        c_nxt = item_cnt(p, it + step, n_items);
-        const SpItem w = sparse_item(p, it, c_cur);
+        c_nxt = WIN ? 0 : item_cnt(p, it + step, n_items);
+        const SpItem w = sparse_item<WIN>(p, it, c_cur);
         const int buf = ii & 1;
         int32_t* pos_s = pos_base + buf * MAX_LIST;
         // ---- the item's list (the buffer's previous item is done with it)
@@ -410,7 +457,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       cp_async_wait<0>();
       if (q_thread && loaded > 0) wait_done(&bars->q_full, (loaded - 1) & 1, p.limit_ns, 302);
     }
-  } else {
+  } else if (warp >= 4) {
     // ============================================ softmax / rescale / epilogue
     const int x = (warp >= 8) ? 1 : 0;  // M tile of this warpgroup
     const int r = threadIdx.x - 128 - 128 * x;
@@ -420,10 +467,10 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     const float sc = KV8 ? 1.f : p.scale_log2;  // KV8 folds the scale into the columns
     int ii = 0, u0 = 0, tx = 0;
     bool ok = true;
-    int c_cur = item_cnt(p, first, n_items), c_nxt = 0;
+    int c_cur = WIN ? 0 : item_cnt(p, first, n_items), c_nxt = 0;
     for (int it = first; it < n_items && ok; it += step, ++ii, c_cur = c_nxt) {
-      c_nxt = item_cnt(p, it + step, n_items);
-      const SpItem w = sparse_item(p, it, c_cur);
+      c_nxt = WIN ? 0 : item_cnt(p, it + step, n_items);
+      const SpItem w = sparse_item<WIN>(p, it, c_cur);
       const int buf = ii & 1;
       const int32_t* pos_s = pos_base + buf * MAX_LIST;
       const int nX = x ? w.nB : w.nt;
@@ -431,7 +478,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       const int i_row = 64 * w.b + mt * p.rows_tok + r / p.G;
       const int hh = w.g * p.G + r % p.G;
       const int i_min = 64 * w.b + mt * p.rows_tok;
-      if (!warp_wait(&bars->list_full[buf], (ii >> 1) & 1, p.limit_ns, abort_flag, 330)) {
+      if (!WIN && !warp_wait(&bars->list_full[buf], (ii >> 1) & 1, p.limit_ns, abort_flag, 330)) {
         ok = false;
         break;
       }
@@ -468,9 +515,14 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
             }
           }
         }
-        // ---- causal mask on listed positions (after any scaling)
+        // ---- mask (after any scaling): the window band, or causal on listed positions
         const int last = j * 128 + 127;
-        if ((last >= w.cnt) || (pos_s[last] > i_min)) {
+        if (WIN) {  // keep i - W < key <= i, key = lo + 128 j + c
+          const int c_hi = i_row - (w.lo + j * 128), c_lo = c_hi - p.window;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > c_hi || c <= c_lo) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+        } else if ((last >= w.cnt) || (pos_s[last] > i_min)) {
           const int4* pv4 = reinterpret_cast<const int4*>(pos_s + j * 128);
 #pragma unroll
           for (int c4 = 0; c4 < 32; ++c4) {
@@ -553,7 +605,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         tc_fence_before();
         mbar_arrive(&bars->p_ready[x]);
       }
-      mbar_arrive(&bars->list_empty[buf]);  // masking is done with this list
+      if (!WIN) mbar_arrive(&bars->list_empty[buf]);  // masking is done with this list
       if (!ok) break;
       // ---- epilogue
       const bool row_live = x == 0 || w.has_b;
@@ -582,6 +634,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         }
         tc_fence_before();
         mbar_arrive(&bars->o_free[x]);
+        if (WIN && p.lse != nullptr)  // natural-log LSE of the row
+          p.lse[static_cast<int64_t>(hh) * p.L + i_row] = (m_used + log2f(l)) * 0.69314718055994530942f;
       } else if (w.nt == 0 && row_live) {
         // an empty list: the rows attend to nothing
         uint4* dst = reinterpret_cast<uint4*>(orow);
