@@ -56,7 +56,8 @@ def algorithmic_work(wl) -> dict:
     # recent positions [e_b - rec, i]
     vis = B * glob + B * (B + 1) / 2.0 + B * (rec - B)   # rec >= B since recent >= block
     sparse = Hq * 4.0 * d * vis.sum()
-    gather = Hkv * (glob + rec).sum() * 2 * 256.0
+    kv_row = 2 * 128 + 8 if getattr(wl, "kv_dtype", "bf16") == "e4m3" else 2 * 256  # K + V row (+ scales)
+    gather = Hkv * (glob + rec).sum() * kv_row
     qo = 2.0 * L * Hq * d * 2
     # sliding-window attention: query i sees min(i + 1, W) keys; Q, K, V read
     # once and O written once
@@ -277,7 +278,7 @@ def cpu_baseline(wl, x, seconds_target: float) -> dict:
 
 # ------------------------------------------------------------- cuda arm --
 
-def select_alone(hs2, torch, shape, q0, k, out, dev, timed, nblk=64):
+def select_alone(hs2, torch, shape, q0, k, ks, out, dev, timed, nblk=64):
     """Kernel (3) by itself on the importance rows of the last `nblk` query
     blocks (the longest rows; a strip larger than L2, so it streams from
     HBM): device time and the row bytes it must read."""
@@ -286,7 +287,7 @@ def select_alone(hs2, torch, shape, q0, k, out, dev, timed, nblk=64):
     n_c = lambda b: max(0, min(shape.L, shape.block * (b + 1)) - shape.recent)
     stride = max(4, (n_c(nb - 1) + 3) // 4 * 4)
     imp = torch.empty((shape.Hkv, nb - b0, stride), dtype=torch.float32, device=dev)
-    hs2.hs2_importance(shape, q0, k, None, out["lse"], b0, nb, imp, stride)
+    hs2.hs2_importance(shape, q0, k, ks, out["lse"], b0, nb, imp, stride)
     ms = timed(lambda: hs2.hs2_topk_select(shape, imp, stride, b0, nb, out["idx"], out["cnt"]), 5)
     moved = shape.Hkv * 4.0 * sum(n_c(b) for b in range(b0, nb) if n_c(b) > shape.topk)
     hs2.hs2_sync()
@@ -298,7 +299,7 @@ def select_alone(hs2, torch, shape, q0, k, out, dev, timed, nblk=64):
 DECODE_BATCHES = (1, 128)   # decode queries per call: one token, and a batch at random positions
 
 
-def decode_rows(hs2, torch, shape, x, k, v, out, dev, timed):
+def decode_rows(hs2, torch, shape, x, k, v, ks, vs, out, dev, timed):
     """Decode-step sparse attention on the prefill's lists: device time per
     call and the listed K/V rows the queries must read (plus Q and O)."""
     res = {}
@@ -314,7 +315,7 @@ def decode_rows(hs2, torch, shape, x, k, v, out, dev, timed):
         o = torch.empty_like(q)
         nbytes = hs2.sparse_decode_workspace_bytes(sh, n)
         ws = torch.empty(nbytes // 4 + 4, dtype=torch.float32, device=dev) if nbytes else None
-        call = lambda: hs2.hs2_sparse_decode(sh, q, pos, k, v, None, None, out["idx"], out["cnt"], o, ws)
+        call = lambda: hs2.hs2_sparse_decode(sh, q, pos, k, v, ks, vs, out["idx"], out["cnt"], o, ws)
         us_eager = 1e3 * timed(call, 50)
         # the same calls replayed from a CUDA graph: device time without the
         # host's per-call cost
@@ -330,7 +331,8 @@ def decode_rows(hs2, torch, shape, x, k, v, out, dev, timed):
         col = torch.arange(lists.shape[-1], device=dev)
         vis = (col[None, None, :] < cnts[..., None]) & (lists >= 0) & (lists <= pos[None, :, None])
         rows = int(vis.sum())
-        moved = rows * 2 * shape.d * k.element_size() + 2 * q.numel() * 2
+        row_bytes = 2 * shape.d * k.element_size() + (8 if k.element_size() == 1 else 0)  # K + V (+ two scales)
+        moved = rows * row_bytes + 2 * q.numel() * 2
         res[f"n{n}"] = {"us_per_call": us, "us_per_call_eager": us_eager, "queries": n, "kv_rows_read": rows, "bytes": moved,
                         "gbs": moved / (us / 1e6) / 1e9, "frac_of_hbm": moved / (us / 1e6) / 1e9 / peaks["hbm_gbs"],
                         "splits_workspace_bytes": nbytes}
@@ -348,16 +350,18 @@ def run_cuda(args, wl, rank, world, dist):
     my = rank_workload(wl, rank, world)
     x = inputs.make_inputs(my, device=dev, with_needles=bool(my.needles))
     q0, k, v = x["q_layers"][0], x["k"], x["v"]
-    shape = hs2.make_shape(q0, k, wl.topk, wl.recent)
+    ks, vs = x.get("k_scale"), x.get("v_scale")  # e4m3 cache: codes + per-token scales
+    fp8_cache = k.dtype == torch.uint8
+    shape = hs2.make_shape(q0, k, wl.topk, wl.recent, kv_dtype=hs2.HS2_KV_E4M3 if fp8_cache else hs2.HS2_KV_BF16)
     out = hs2.alloc_outputs(shape, q0)
     o_sp = [torch.empty_like(q) for q in x["q_layers"][1:]]
     stream = torch.cuda.current_stream()
 
     def step():
-        hs2.hs2_full_attn_select(shape, q0, k, v, None, None, out["o"], out["lse"], out["idx"], out["cnt"],
+        hs2.hs2_full_attn_select(shape, q0, k, v, ks, vs, out["o"], out["lse"], out["idx"], out["cnt"],
                                  out["workspace"], stream)
         for ql, ol in zip(x["q_layers"][1:], o_sp):
-            hs2.hs2_sparse_attn(shape, ql, k, v, None, None, out["idx"], out["cnt"], ol, stream)
+            hs2.hs2_sparse_attn(shape, ql, k, v, ks, vs, out["idx"], out["cnt"], ol, stream)
 
     def barrier():
         if dist is not None:
@@ -408,25 +412,25 @@ def run_cuda(args, wl, rank, world, dist):
         fp8 = {"ms": qk_ms, "gbs": moved / (qk_ms / 1e3) / 1e9, "frac_of_hbm": moved / (qk_ms / 1e3) / 1e9 /
                measured_peaks()["hbm_gbs"], "bytes": moved}
         del codes, kscale
-    fa_ms = timed(lambda: hs2.hs2_attn_fwd(shape, q0, k, v, None, None, out["o"], out["lse"], stream), n_stage)
-    sp_ms = timed(lambda: hs2.hs2_sparse_attn(shape, x["q_layers"][1], k, v, None, None, out["idx"], out["cnt"],
+    fa_ms = timed(lambda: hs2.hs2_attn_fwd(shape, q0, k, v, ks, vs, out["o"], out["lse"], stream), n_stage)
+    sp_ms = timed(lambda: hs2.hs2_sparse_attn(shape, x["q_layers"][1], k, v, ks, vs, out["idx"], out["cnt"],
                                               o_sp[0], stream), n_stage) if o_sp else 0.0
-    fs_ms = timed(lambda: hs2.hs2_full_attn_select(shape, q0, k, v, None, None, out["o"], out["lse"], out["idx"],
+    fs_ms = timed(lambda: hs2.hs2_full_attn_select(shape, q0, k, v, ks, vs, out["o"], out["lse"], out["idx"],
                                                    out["cnt"], out["workspace"], stream), n_stage)
     blk_ms = timed(lambda: hs2.hs2_full_attn_select_blocks(shape, q0, k, v, None, None, out["o"], out["lse"],
                                                            out["idx"], out["cnt"], out["workspace"], stream),
                    n_stage) if wl.topk % 64 == 0 and k.dtype == torch.bfloat16 else None
     swa_ms = timed(lambda: hs2.hs2_swa_attn(shape, q0, k, v, SWA_WINDOW, out["o"], None, stream),
                    n_stage) if k.dtype == torch.bfloat16 else None
-    decode = decode_rows(hs2, torch, shape, x, k, v, out, dev, timed) if o_sp else None
-    select = select_alone(hs2, torch, shape, q0, k, out, dev, timed)
+    decode = decode_rows(hs2, torch, shape, x, k, v, ks, vs, out, dev, timed) if o_sp else None
+    select = select_alone(hs2, torch, shape, q0, k, ks, out, dev, timed)
     hs2.hs2_sync(stream)
 
     # ---- end to end from pinned host buffers: every step copies its inputs in
     # and every output back, through the same C ABI calls, with the copies
     # overlapped with compute on separate streams (PrefillPipeline)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not fp8_cache:  # the end-to-end runner takes a bf16 cache
         from token_level_sparse_causal_b200.pipeline import PrefillPipeline
         h_q = [t.cpu().pin_memory() for t in x["q_layers"]]
         h_k, h_v = k.cpu().pin_memory(), v.cpu().pin_memory()
@@ -463,7 +467,8 @@ def run_cuda(args, wl, rank, world, dist):
         "metric": METRIC, "value": job_throughput(wl.L, world, ms), "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "p50_ms": float(np.percentile(per, 50)), "p99_ms": float(np.percentile(per, 99)),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 Q, e4m3 K/V (f16 MMA)" if fp8_cache else "bf16",
         "data": "synthetic (seeded; K from a 64-component Gaussian mixture, std 0.3)",
         "config": {"workload": wl.name, "L": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
                    "layers": f"1 full + {wl.n_sparse} sparse", "topk": wl.topk, "recent": wl.recent,

@@ -315,18 +315,24 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           for (int half = 0; half < 2; ++half) {  // 0: K, 1: V
             const uint8_t* base8 = half ? vb8 : kb8;
             const float* scale = half ? p.vsc : p.ksc;
-#pragma unroll 4
+            // every row's codes and scale in flight before any is converted
+            uint4 raw[16];
+            float sgv[16];
+#pragma unroll
+            for (int it = 0; it < 16; ++it) {
+              const int pj = j * 128 + rsub + 8 * it;
+              raw[it] = make_uint4(0, 0, 0, 0);
+              sgv[it] = 0.f;
+              if (pj < p.L) {
+                raw[it] = ld_nc_v4(base8 + static_cast<int64_t>(pj) * p.kv_tok);
+                sgv[it] = scale[static_cast<int64_t>(pj) * p.Hkv + g];
+              }
+            }
+#pragma unroll
             for (int it = 0; it < 16; ++it) {
               const int r = rsub + 8 * it;
-              const int pj = j * 128 + r;
-              const bool valid = pj < p.L;
-              uint4 raw = make_uint4(0, 0, 0, 0);
-              float sg = 0.f;
-              if (valid) {
-                raw = ld_nc_v4(base8 + static_cast<int64_t>(pj) * p.kv_tok);
-                sg = scale[static_cast<int64_t>(pj) * p.Hkv + g];
-              }
-              const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+              const float sg = sgv[it];
+              const uint32_t w[4] = {raw[it].x, raw[it].y, raw[it].z, raw[it].w};
               uint32_t f[8];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {

@@ -384,19 +384,24 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
             for (int half = 0; half < 2; ++half) {  // 0: K, 1: V
               const uint8_t* base8 = half ? vb8 : kb8;
               const float* scale = half ? p.vsc : p.ksc;
-#pragma unroll 4
+              // every row's codes and scale in flight before any is converted
+              uint4 raw[16];
+              float sgv[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int pj = pos_s[j * 128 + rsub + 8 * i];
+                raw[i] = make_uint4(0, 0, 0, 0);
+                sgv[i] = 0.f;
+                if (pj >= 0) {
+                  raw[i] = ld_nc_v4(base8 + static_cast<int64_t>(pj) * p.kv_tok);
+                  sgv[i] = scale[static_cast<int64_t>(pj) * p.Hkv + w.g];
+                }
+              }
+#pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const int r = rsub + 8 * i;
-                const int gi = j * 128 + r;
-                const int pj = pos_s[gi];
-                const bool valid = pj >= 0;
-                uint4 raw = make_uint4(0, 0, 0, 0);
-                float sg = 0.f;
-                if (valid) {
-                  raw = ld_nc_v4(base8 + static_cast<int64_t>(pj) * p.kv_tok);
-                  sg = scale[static_cast<int64_t>(pj) * p.Hkv + w.g];
-                }
-                const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+                const float sg = sgv[i];
+                const uint32_t wd[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
                 uint32_t f[8];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
