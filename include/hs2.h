@@ -93,6 +93,12 @@ typedef struct hs2_shape {
  *   `workspace` (16-byte aligned); it must be at least
  *   Hkv * roundup(L - recent, 64) * 4 bytes (one block per strip), else
  *   HS2_ERR_WORKSPACE.  The workspace holds no state between calls.
+ *   With an e4m3 cache the recommended size also holds an f16 copy of the
+ *   layer's K and V (2 * L * Hkv * 128 * 2 bytes, plus Hkv * roundup(L, 128)
+ *   * 4 bytes of K scales and 768 bytes of alignment), taken from the end of
+ *   the workspace whenever it fits beside the minimum: the cache is then
+ *   converted once instead of inside every tile load of the attention and
+ *   importance kernels.  Results are identical either way.
  */
 int hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, const void* v,
                          const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,

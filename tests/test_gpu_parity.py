@@ -445,6 +445,37 @@ def test_fp8_importance_select_and_sparse_match_oracle(L, Hq, Hkv):
     assert all(H.guards_intact(bb) for bb in r["bases"])
 
 
+@pytest.mark.parametrize("L,Hq,Hkv", [(2368, 8, 1), (1088, 8, 2), (3072, 16, 2)])
+def test_fp8_layer_copy_equals_in_kernel_conversion(L, Hq, Hkv):
+    """hs2_full_attn_select converts an e4m3 cache to f16 once per layer when
+    the workspace also holds that copy, and inside kernels (1) and (2)
+    otherwise: both must give the same bits (O, LSE, lists), and the same O /
+    LSE as hs2_attn_fwd, which always converts in the kernel."""
+    wl = _fp8_wl(L, Hq, Hkv, n_sparse=0, seed=37, topk=1000)
+    xd = H.to_dev(inputs.make_inputs(wl), DEV)
+    shape = H.shape_of(wl, xd)
+    q0, k, v, ks, vs = xd["q_layers"][0], xd["k"], xd["v"], xd["k_scale"], xd["v_scale"]
+    nb = L // 64
+    ws_min = Hkv * ((L - 128 + 63) // 64 * 64) * 4
+    ws_rec = hs2.workspace_bytes(shape)
+    assert ws_rec >= ws_min + 2 * L * Hkv * 128 * 2  # room for the f16 copy
+    outs = []
+    for nbytes in (ws_min, ws_rec):
+        o, lse = torch.empty_like(q0), torch.empty((Hq, L), device=DEV, dtype=torch.float32)
+        idx = torch.empty((Hkv, nb, wl.topk + wl.recent), device=DEV, dtype=torch.int32)
+        cnt = torch.empty((Hkv, nb), device=DEV, dtype=torch.int32)
+        ws = torch.empty(nbytes // 4, device=DEV, dtype=torch.float32)
+        hs2.hs2_full_attn_select(shape, q0, k, v, ks, vs, o, lse, idx, cnt, ws)
+        hs2.hs2_sync()
+        outs.append((o, lse, idx, cnt))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+    o1, lse1 = torch.empty_like(q0), torch.empty((Hq, L), device=DEV, dtype=torch.float32)
+    hs2.hs2_attn_fwd(shape, q0, k, v, ks, vs, o1, lse1)
+    hs2.hs2_sync()
+    assert torch.equal(o1, outs[1][0]) and torch.equal(lse1, outs[1][1])
+
+
 # -------------------------------------------------- device-side failures --
 
 def test_bounded_wait_reports_timeout_and_context_survives():

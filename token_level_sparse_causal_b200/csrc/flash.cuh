@@ -2,27 +2,33 @@
 // the sliding window's persistent kernel in sparse_attn.cuh is built on the
 // same pipeline):
 //
-//   FLASH_DENSE  -- kernel (1): causal grouped-query attention of the full
-//                   layer, one CTA per (pair of 128-query tiles, query head),
-//                   K/V tiles of 128 keys streamed by TMA; writes O and the
-//                   per-query natural-log LSE.  (HySparse2 architecture
-//                   summary, ablation paragraph: the full layer's complete
-//                   scores; SHARP walk-through, section 1.1:
-//                   softmax(Q K^T / sqrt(d)) V.)
+// Kernel (1): causal grouped-query attention of the full layer, one CTA per
+// (pair of 128-query tiles, query head), K/V tiles of 128 keys streamed
+// through shared memory; writes O and the per-query natural-log LSE.
+// (HySparse2 architecture summary, ablation paragraph: the full layer's
+// complete scores; SHARP walk-through, section 1.1: softmax(Q K^T / sqrt(d)) V.)
 //
 // CTA = 12 warps:
-//   warp 0      TMA: Q tiles, K/V tiles (bf16 cache)
+//   warp 0      TMA: Q tiles, K/V tiles (bf16 cache, or the f16 copy of an
+//               FP8 cache with its K column scales)
 //   warp 1      TMEM allocation; one thread issues every tcgen05.mma
-//   warps 2-3   with an FP8 cache: convert Q to f16 in place, then load,
-//               convert and scale every K/V tile
+//   warps 2-3   with an FP8 cache: convert Q to f16 in place; when reading
+//               the e4m3 codes directly, also load, convert and scale every
+//               K/V tile
 //   warps 4-7   softmax / rescale / epilogue of query tile A (thread r <-> row r)
 //   warps 8-11  the same for query tile B
 //
-// FP8 e4m3 cache (KV8): every e4m3 value is an f16 value, so codes are
-// converted exactly to f16 (one cvt per pair), Q is converted bf16 -> f16 in
-// shared memory after its TMA load, and all MMAs run kind::f16 on f16
-// operands.  The per-token K scale (times log2(e)/sqrt(d)) multiplies the S
-// columns in fp32; the V scale is folded into the converted V rows.
+// FP8 e4m3 cache: every e4m3 value is an f16 value, so codes convert exactly
+// to f16, Q is converted bf16 -> f16 in shared memory after its TMA load, and
+// all MMAs run kind::f16 on f16 operands.  The per-token K scale (times
+// log2(e)/sqrt(d)) multiplies the S columns in fp32; the V scale is folded
+// into the f16 V rows.  Two ways to get the f16 tiles, same values:
+//   KVM_E4M3  warps 2-3 load the codes and convert every tile in the kernel
+//             (no scratch memory);
+//   KVM_F16   the cache was converted once for the layer (dequant_kv_kernel)
+//             and warp 0 loads f16 tiles by TMA plus each tile's 128 column
+//             scales by a bulk copy -- the conversion is not repeated for
+//             every query head and query tile that reads the tile.
 // (HySparse2 architecture summary, cost paragraph: FP8 KV cache.)
 //
 // Tensor memory (512 columns): S_A [0,128), S_B [128,256), O_A [256,384),
@@ -55,7 +61,10 @@ constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
 constexpr uint32_t IDESC_S_F16 = idesc_f16_f32(128, 128, 0, 0);
 constexpr uint32_t IDESC_PV_F16 = idesc_f16_f32(128, 128, 0, 1);
-constexpr int FLASH_DENSE = 0;
+// K/V cache modes of the dense kernels
+constexpr int KVM_BF16 = 0;  // bf16 cache, TMA
+constexpr int KVM_E4M3 = 1;  // e4m3 codes, converted in the kernel
+constexpr int KVM_F16 = 2;   // f16 copy of an e4m3 cache (+ K column scales), TMA
 constexpr uint32_t FLAG_SKIP_LOADS = 1u;
 constexpr int MAX_LIST = 4096;
 
@@ -71,6 +80,8 @@ struct FlashParams {
   const uint8_t* v8;
   const float* ksc;
   const float* vsc;
+  const float* kcol;  // KVM_F16: K scale x log2(e)/sqrt(d), [Hkv][kcol_stride]
+  int kcol_stride;    // L rounded up to 128
   int64_t kv_tok, kv_head;
   const int32_t* idx;
   const int32_t* cnt;
@@ -126,11 +137,12 @@ __device__ __forceinline__ bool wait_done(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
-template <int MODE, bool KV8>
+template <int KVM>
 __global__ void __launch_bounds__(FL_THREADS, 1)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const FlashParams p) {
-  static_assert(MODE == FLASH_DENSE, "one mode: causal attention + LSE");
+  constexpr bool KV8 = KVM != KVM_BF16;   // f16 operands, K column scales
+  constexpr bool CONV = KVM == KVM_E4M3;  // K/V tiles converted by warps 2-3
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   FlashBars* bars = reinterpret_cast<FlashBars*>(smem + FL_BAR_OFF);
@@ -156,7 +168,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
   const bool has_b = nB > 0;
 
   if (threadIdx.x == 0) {
-    const uint32_t kv_arrivals = KV8 ? 64u : 1u;
+    const uint32_t kv_arrivals = CONV ? 64u : 1u;
     mbar_init(&bars->q_raw, 1);
     mbar_init(&bars->q_full, KV8 ? 64u : 1u);
     for (int s = 0; s < FL_STAGES; ++s) {
@@ -194,7 +206,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         tma_load_3d(qd, &tmQ, qbar, 0, h, (2 * pair + x) * 128);
         tma_load_3d(qd + HALF_BYTES, &tmQ, qbar, 64, h, (2 * pair + x) * 128);
       }
-      if (!KV8) {
+      if (!CONV) {
         int last = -1;
         for (int j = 0; j < n; ++j) {
           const int u = j;  // position in this CTA's key-tile stream
@@ -203,7 +215,9 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
               !mbar_wait(&bars->empty[s], ((u / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 101))
             break;
           uint8_t* kd = smem + FL_KV_OFF + s * 2 * TILE_BYTES;
-          mbar_arrive_expect_tx(&bars->full_k[s], TILE_BYTES);
+          mbar_arrive_expect_tx(&bars->full_k[s], TILE_BYTES + (KV8 ? 512u : 0u));
+          if (KV8) bulk_load(ksc_s + s * 128, p.kcol + static_cast<int64_t>(g) * p.kcol_stride + j * 128, 512u,
+                             &bars->full_k[s]);
           tma_load_3d(kd, &tmK, &bars->full_k[s], 0, g, j * 128);
           tma_load_3d(kd + HALF_BYTES, &tmK, &bars->full_k[s], 64, g, j * 128);
           mbar_arrive_expect_tx(&bars->full_v[s], TILE_BYTES);
@@ -305,7 +319,7 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         const int rsub = pt >> 3, c8 = pt & 7;
         const uint8_t* kb8 = p.k8 + static_cast<int64_t>(g) * p.kv_head + c8 * 16;
         const uint8_t* vb8 = p.v8 + static_cast<int64_t>(g) * p.kv_head + c8 * 16;
-        for (int j = 0; j < n; ++j) {
+        for (int j = 0; j < (CONV ? n : 0); ++j) {  // KVM_F16: K/V tiles come by TMA
           const int s = j % FL_STAGES;
           if (j >= FL_STAGES &&
               !mbar_wait(&bars->empty[s], ((j / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 142))

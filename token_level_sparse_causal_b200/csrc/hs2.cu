@@ -130,8 +130,66 @@ int set_smem(K kernel, uint32_t bytes) {
 
 // ------------------------------------------------------------- launches --
 
+// The f16 copy of an e4m3 cache made once per layer by dequant_kv_kernel
+// (inside a caller workspace): K and V [L][Hkv][128] f16, K column scales
+// [Hkv][Lp].
+struct DequantBuf {
+  uint16_t* kf;
+  uint16_t* vf;
+  float* kcol;
+  int Lp;
+};
+
+int kcol_stride(const hs2_shape* s) { return (s->L + 127) / 128 * 128; }
+
+size_t dequant_bytes(const hs2_shape* s) {
+  const size_t kv = static_cast<size_t>(s->L) * s->Hkv * HD * 2u;
+  return 2 * kv + static_cast<size_t>(s->Hkv) * kcol_stride(s) * 4u + 3 * 256;
+}
+
+// Carves a DequantBuf from [base, base + dequant_bytes(s)).
+DequantBuf dequant_carve(const hs2_shape* s, uint8_t* base) {
+  auto up = [](uint8_t* x) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(x) + 255) & ~static_cast<uintptr_t>(255));
+  };
+  const size_t kv = static_cast<size_t>(s->L) * s->Hkv * HD * 2u;
+  DequantBuf d{};
+  uint8_t* x = up(base);
+  d.kf = reinterpret_cast<uint16_t*>(x);
+  x = up(x + kv);
+  d.vf = reinterpret_cast<uint16_t*>(x);
+  x = up(x + kv);
+  d.kcol = reinterpret_cast<float*>(x);
+  d.Lp = kcol_stride(s);
+  return d;
+}
+
+int launch_dequant(const hs2_shape* s, const void* k, const void* v, const float* ks, const float* vs,
+                   const DequantBuf& d, cudaStream_t st) {
+  DequantParams p{};
+  p.L = s->L;
+  p.Hkv = s->Hkv;
+  p.Lp = d.Lp;
+  p.k8 = static_cast<const uint8_t*>(k);
+  p.v8 = static_cast<const uint8_t*>(v);
+  p.kv_tok = s->kv_tok_stride;
+  p.kv_head = s->kv_head_stride;
+  p.ksc = ks;
+  p.vsc = vs;
+  p.kf = d.kf;
+  p.vf = d.vf;
+  p.kcol = d.kcol;
+  p.scale_log2 = scale_log2(s->d);
+  const int64_t rows = static_cast<int64_t>(d.Lp) * s->Hkv;
+  const int64_t blocks = std::min<int64_t>((rows + 31) / 32, static_cast<int64_t>(sm_count()) * 8);
+  dequant_kv_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(p);
+  return launched();
+}
+
+// Kernel (1).  dq: the layer's f16 copy of an e4m3 cache (KVM_F16), or null
+// to read the cache itself (bf16 by TMA, or e4m3 converted in the kernel).
 int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void* v, const float* ks,
-                    const float* vs, void* o, float* lse, cudaStream_t st) {
+                    const float* vs, void* o, float* lse, cudaStream_t st, const DequantBuf* dq = nullptr) {
   const bool kv8 = s->kv_dtype == HS2_KV_E4M3;
   CUtensorMap mq, mk, mv;
   int rc;
@@ -139,6 +197,9 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
   if (!kv8) {
     if ((rc = make_map(&mk, k, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
     if ((rc = make_map(&mv, v, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+  } else if (dq) {
+    if ((rc = make_map(&mk, dq->kf, s->L, s->Hkv, int64_t(s->Hkv) * HD, HD, 1, 128))) return rc;
+    if ((rc = make_map(&mv, dq->vf, s->L, s->Hkv, int64_t(s->Hkv) * HD, HD, 1, 128))) return rc;
   } else {
     mk = mq;
     mv = mq;
@@ -148,6 +209,10 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
   p.v8 = static_cast<const uint8_t*>(v);
   p.ksc = ks;
   p.vsc = vs;
+  if (dq) {
+    p.kcol = dq->kcol;
+    p.kcol_stride = dq->Lp;
+  }
   p.kv_tok = s->kv_tok_stride;
   p.kv_head = s->kv_head_stride;
   p.L = s->L;
@@ -164,14 +229,18 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
   p.limit_ns = g_wait_limit_ns;
   p.flags = g_flags;
   const unsigned grid = static_cast<unsigned>(p.npairs * s->Hq);
-  if (kv8) {
-    static int attr8 = set_smem(flash_fwd_kernel<FLASH_DENSE, true>, FL_SMEM_KV8);
+  if (kv8 && dq) {
+    static int attr16 = set_smem(flash_fwd_kernel<KVM_F16>, FL_SMEM_KV8);
+    if (attr16) return attr16;
+    flash_fwd_kernel<KVM_F16><<<grid, FL_THREADS, FL_SMEM_KV8, st>>>(mq, mk, mv, p);
+  } else if (kv8) {
+    static int attr8 = set_smem(flash_fwd_kernel<KVM_E4M3>, FL_SMEM_KV8);
     if (attr8) return attr8;
-    flash_fwd_kernel<FLASH_DENSE, true><<<grid, FL_THREADS, FL_SMEM_KV8, st>>>(mq, mk, mv, p);
+    flash_fwd_kernel<KVM_E4M3><<<grid, FL_THREADS, FL_SMEM_KV8, st>>>(mq, mk, mv, p);
   } else {
-    static int attr = set_smem(flash_fwd_kernel<FLASH_DENSE, false>, FL_SMEM_DENSE);
+    static int attr = set_smem(flash_fwd_kernel<KVM_BF16>, FL_SMEM_DENSE);
     if (attr) return attr;
-    flash_fwd_kernel<FLASH_DENSE, false><<<grid, FL_THREADS, FL_SMEM_DENSE, st>>>(mq, mk, mv, p);
+    flash_fwd_kernel<KVM_BF16><<<grid, FL_THREADS, FL_SMEM_DENSE, st>>>(mq, mk, mv, p);
   }
   return launched();
 }
@@ -317,17 +386,19 @@ int launch_decode(const hs2_shape* s, const void* q, const int32_t* positions, i
 
 int n_cand(const hs2_shape* s, int b) { return std::max(0, std::min(s->L, 64 * (b + 1)) - s->recent); }
 
-template <int G, bool KV8>
+template <int G, int KVM>
 int launch_importance_g(const CUtensorMap& mq, const CUtensorMap& mk, const ImpParams& p, dim3 grid,
                         cudaStream_t st) {
-  static int attr = set_smem(importance_kernel<G, KV8>, imp_smem_bytes(G));
+  static int attr = set_smem(importance_kernel<G, KVM>, imp_smem_bytes(G));
   if (attr) return attr;
-  importance_kernel<G, KV8><<<grid, IMP_THREADS, imp_smem_bytes(G), st>>>(mq, mk, p);
+  importance_kernel<G, KVM><<<grid, IMP_THREADS, imp_smem_bytes(G), st>>>(mq, mk, p);
   return launched();
 }
 
+// Kernel (2) for blocks [b0, b1).  dq as in launch_attn_fwd.
 int launch_importance(const hs2_shape* s, const void* q, const void* k, const float* ks, const float* lse, int b0,
-                      int b1, float* imp, int64_t row_stride, int skip_le, cudaStream_t st) {
+                      int b1, float* imp, int64_t row_stride, int skip_le, cudaStream_t st,
+                      const DequantBuf* dq = nullptr) {
   const bool kv8 = s->kv_dtype == HS2_KV_E4M3;
   const int G = s->Hq / s->Hkv;
   const int longest = n_cand(s, b1 - 1);
@@ -337,6 +408,8 @@ int launch_importance(const hs2_shape* s, const void* q, const void* k, const fl
   if ((rc = make_map(&mq, q, s->L, s->Hq, s->q_tok_stride, s->q_head_stride, G, 64))) return rc;
   if (!kv8) {
     if ((rc = make_map(&mk, k, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 128))) return rc;
+  } else if (dq) {
+    if ((rc = make_map(&mk, dq->kf, s->L, s->Hkv, int64_t(s->Hkv) * HD, HD, 1, 128))) return rc;
   } else {
     mk = mq;
   }
@@ -360,13 +433,17 @@ int launch_importance(const hs2_shape* s, const void* q, const void* k, const fl
   p.limit_ns = g_wait_limit_ns;
   p.flags = g_flags;
   const dim3 grid(static_cast<unsigned>((longest + IMP_CK - 1) / IMP_CK), static_cast<unsigned>(s->Hkv * (b1 - b0)));
-  switch (G * 2 + (kv8 ? 1 : 0)) {
-    case 4: return launch_importance_g<2, false>(mq, mk, p, grid, st);
-    case 5: return launch_importance_g<2, true>(mq, mk, p, grid, st);
-    case 8: return launch_importance_g<4, false>(mq, mk, p, grid, st);
-    case 9: return launch_importance_g<4, true>(mq, mk, p, grid, st);
-    case 16: return launch_importance_g<8, false>(mq, mk, p, grid, st);
-    case 17: return launch_importance_g<8, true>(mq, mk, p, grid, st);
+  const int kvm = !kv8 ? KVM_BF16 : (dq ? KVM_F16 : KVM_E4M3);
+  switch (G * 4 + kvm) {
+    case 8: return launch_importance_g<2, KVM_BF16>(mq, mk, p, grid, st);
+    case 9: return launch_importance_g<2, KVM_E4M3>(mq, mk, p, grid, st);
+    case 10: return launch_importance_g<2, KVM_F16>(mq, mk, p, grid, st);
+    case 16: return launch_importance_g<4, KVM_BF16>(mq, mk, p, grid, st);
+    case 17: return launch_importance_g<4, KVM_E4M3>(mq, mk, p, grid, st);
+    case 18: return launch_importance_g<4, KVM_F16>(mq, mk, p, grid, st);
+    case 32: return launch_importance_g<8, KVM_BF16>(mq, mk, p, grid, st);
+    case 33: return launch_importance_g<8, KVM_E4M3>(mq, mk, p, grid, st);
+    case 34: return launch_importance_g<8, KVM_F16>(mq, mk, p, grid, st);
     default: return HS2_ERR_UNSUPPORTED;
   }
 }
@@ -421,11 +498,14 @@ size_t min_workspace(const hs2_shape* s) {
 
 constexpr size_t kStripCap = size_t(64) << 20;  // keep one strip L2-resident
 
+// Strips in as few launches as the L2 cap allows; with an e4m3 cache, plus
+// room for the layer's f16 copy (dequant_bytes).
 size_t recommended_workspace(const hs2_shape* s) {
   size_t whole = 0;
   const int nb = s->L / 64;
   for (int b = 0; b < nb; ++b) whole += static_cast<size_t>(s->Hkv) * strip_stride(s, b) * 4u;
-  return std::max(min_workspace(s), std::min(whole, kStripCap));
+  const size_t strips = std::max(min_workspace(s), std::min(whole, kStripCap));
+  return strips + (s->kv_dtype == HS2_KV_E4M3 ? dequant_bytes(s) : 0u);
 }
 
 // Scratch for hs2_full_attn_select_static: the importance strips of callers
@@ -598,10 +678,21 @@ int full_attn_select_impl(const hs2_shape* shape, const void* q, const void* k, 
   if ((rc = check_kv(shape, k, v, k_scale, v_scale))) return rc;
   if (!q || !o || !lse || !idx || !cnt) return HS2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || !aligned16(workspace)) return HS2_ERR_UNSUPPORTED;
-  const size_t ws = *workspace_bytes;
+  size_t ws = *workspace_bytes;
   if (ws < min_workspace(shape)) return HS2_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((rc = launch_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, st))) return rc;
+  // An e4m3 cache is converted to f16 once for the layer when the workspace
+  // also holds that copy (at its end); otherwise kernels (1) and (2) convert
+  // the tiles they load.  The results are the same.
+  DequantBuf dqb{};
+  const DequantBuf* dq = nullptr;
+  if (shape->kv_dtype == HS2_KV_E4M3 && ws >= min_workspace(shape) + dequant_bytes(shape)) {
+    ws -= dequant_bytes(shape);
+    dqb = dequant_carve(shape, static_cast<uint8_t*>(workspace) + ws);
+    dq = &dqb;
+    if ((rc = launch_dequant(shape, k, v, k_scale, v_scale, dqb, st))) return rc;
+  }
+  if ((rc = launch_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, st, dq))) return rc;
 
   // Strips of query blocks.  Blocks whose candidates all fit in the top-k
   // need no importance; the rest are grouped so that a strip's rows
@@ -617,7 +708,7 @@ int full_attn_select_impl(const hs2_shape* shape, const void* q, const void* k, 
     } else {
       while (b1 < nb && static_cast<size_t>(shape->Hkv) * (b1 + 1 - b) * strip_stride(shape, b1) * 4u <= ws) ++b1;
       const int64_t stride = strip_stride(shape, b1 - 1);
-      if ((rc = launch_importance(shape, q, k, k_scale, lse, b, b1, imp, stride, shape->topk, st))) return rc;
+      if ((rc = launch_importance(shape, q, k, k_scale, lse, b, b1, imp, stride, shape->topk, st, dq))) return rc;
       if ((rc = launch_select(shape, imp, stride, b, b1, idx, cnt, st, blocks))) return rc;
     }
     b = b1;

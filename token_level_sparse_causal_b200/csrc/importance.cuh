@@ -25,9 +25,11 @@
 // hs2_importance reproduces exactly what the selection saw).  Arguments and
 // sums use packed f32x2 FMA/ADD; a quarter of the exponentials run on the FMA
 // pipes (exp2_fma3), the rest on the MUFU unit -- the share measured fastest.
-// FP8 e4m3 cache (KV8): warps 2-3 convert the Q block to f16 in place and
-// convert each K tile exactly from e4m3 to f16 (MMAs run kind::f16); each
-// key's fp32 scale multiplies its row of scores in the epilogue.
+// FP8 e4m3 cache: warps 2-3 convert the Q block to f16 in place, and the K
+// tiles are f16 (MMAs run kind::f16): either converted exactly from the codes
+// by warps 2-3 (KVM_E4M3) or loaded by TMA from the layer's f16 copy
+// (KVM_F16, see dequant_kv_kernel); each key's fp32 scale multiplies its row
+// of scores in the epilogue.
 // Work item = (KV head, block, chunk of IMP_CK keys); the grid is
 // (chunks of the longest row of the strip) x (Hkv * blocks).
 #pragma once
@@ -79,10 +81,12 @@ __host__ __device__ constexpr uint32_t imp_smem_bytes(int G) {
   return imp_part_off(G) + (IMP_GROUPS - 1) * 2u * 128u * 4u + 1024u;
 }
 
-template <int G, bool KV8>
+template <int G, int KVM>
 __global__ void __launch_bounds__(IMP_THREADS, 1)
     importance_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const ImpParams p) {
+  constexpr bool KV8 = KVM != KVM_BF16;   // f16 operands, per-key scales
+  constexpr bool CONV = KVM == KVM_E4M3;  // K tiles converted by warps 2-3
   constexpr int NQ = 64 * G;                    // query-head rows of a block
   constexpr int NSUB = (NQ < 256) ? NQ : 256;   // MMA N per sub-tile
   constexpr int SUBS = NQ / NSUB;
@@ -113,7 +117,7 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
     mbar_init(&bars->q_raw, 1);
     mbar_init(&bars->q_full, KV8 ? 64u : 1u);
     for (int s = 0; s < IMP_STAGES; ++s) {
-      mbar_init(&bars->k_full[s], KV8 ? 64u : 1u);
+      mbar_init(&bars->k_full[s], CONV ? 64u : 1u);
       mbar_init(&bars->k_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -149,7 +153,7 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
       tma_load_3d(smem, &tmQ, qbar, 0, g * G, 64 * b);
       tma_load_3d(smem + QHALF, &tmQ, qbar, 64, g * G, 64 * b);
       int last = -1;
-      for (int t = 0; t < (KV8 ? 0 : ntiles); ++t) {
+      for (int t = 0; t < (CONV ? 0 : ntiles); ++t) {
         const int s = t % IMP_STAGES;
         if (t >= IMP_STAGES &&
             !mbar_wait(&bars->k_empty[s], ((t / IMP_STAGES) - 1) & 1, p.limit_ns, abort_flag, 201))
@@ -200,8 +204,9 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
       wait_done(&bars->fin, 0, p.limit_ns, 214);
     }
   } else if (warp < 4) {
-    // KV8: convert the Q block to f16 in place, then load, convert (exactly,
-    // e4m3 -> f16) and store every K tile; 8 threads per 128-byte code row.
+    // FP8 cache: convert the Q block to f16 in place; KVM_E4M3 then loads,
+    // converts (exactly, e4m3 -> f16) and stores every K tile, 8 threads per
+    // 128-byte code row.
     if (KV8 && !(p.flags & FLAG_SKIP_LOADS)) {
       const int pt = threadIdx.x - 64;
       if (mbar_wait(&bars->q_raw, 0, p.limit_ns, abort_flag, 241)) {
@@ -213,7 +218,7 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
         mbar_arrive(&bars->q_full);
         const int rsub = pt >> 3, c8 = pt & 7;
         const uint8_t* kb8 = p.k8 + static_cast<int64_t>(g) * p.kv_head + c8 * 16;
-        for (int t = 0; t < ntiles; ++t) {
+        for (int t = 0; t < (CONV ? ntiles : 0); ++t) {  // KVM_F16: K tiles come by TMA
           const int s = t % IMP_STAGES;
           if (t >= IMP_STAGES &&
               !mbar_wait(&bars->k_empty[s], ((t / IMP_STAGES) - 1) & 1, p.limit_ns, abort_flag, 242))

@@ -79,3 +79,86 @@ __global__ void __launch_bounds__(256) quantize_kv_kernel(const QuantParams p) {
 }
 
 }  // namespace hs2
+
+namespace hs2 {
+
+// Once-per-layer dequantisation of the e4m3 cache for the dense passes.
+//
+// The full-attention kernel and the importance pass read every K/V tile of a
+// KV head once per query tile and query head; converting the codes inside
+// those kernels repeats the same conversion G * (tiles before it) times and
+// competes with the softmax for the conversion units.  This pass converts the
+// cache once into f16 buffers the dense kernels load by TMA, with exactly the
+// arithmetic of the in-kernel converters:
+//   kf[t][g][:]  = f16(code)                (exact: every e4m3 value is an f16)
+//   vf[t][g][:]  = f16(code) * f16(vscale)  (one f16 multiply, as in the gather)
+//   kcol[g][t]   = kscale[t][g] * log2(e)/sqrt(d)   (fp32; 0 for L <= t < Lp)
+// Memory-bound: 2 x 128 B + 8 B read, 2 x 256 B + 4 B written per row.
+struct DequantParams {
+  int L, Hkv, Lp;  // Lp: kcol row stride (L rounded up to the key tile)
+  const uint8_t* k8;
+  const uint8_t* v8;
+  int64_t kv_tok, kv_head;  // bytes
+  const float* ksc;         // [L][Hkv]
+  const float* vsc;
+  uint16_t* kf;  // f16 bits, [L][Hkv][128] contiguous
+  uint16_t* vf;
+  float* kcol;  // [Hkv][Lp]
+  float scale_log2;
+};
+
+// Eight threads per (token, head) row, 16 codes of K and 16 of V each; every
+// thread issues the loads of ROWS rows before converting any.
+__global__ void __launch_bounds__(256) dequant_kv_kernel(const DequantParams p) {
+  constexpr int ROWS = 4;  // row steps per thread and iteration
+  const int64_t rows = static_cast<int64_t>(p.Lp) * p.Hkv;
+  const int c8 = threadIdx.x & 7;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 3);
+  for (int64_t r0 = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 3) + (threadIdx.x >> 3); r0 < rows;
+       r0 += stride * ROWS) {
+    uint4 rk[ROWS], rv[ROWS];
+    float sk[ROWS], sv[ROWS];
+#pragma unroll
+    for (int u = 0; u < ROWS; ++u) {
+      const int64_t row = r0 + u * stride;
+      const int t = static_cast<int>(row / p.Hkv), g = static_cast<int>(row % p.Hkv);
+      rk[u] = rv[u] = make_uint4(0, 0, 0, 0);
+      sk[u] = sv[u] = 0.f;
+      if (row < rows && t < p.L) {
+        const int64_t off = static_cast<int64_t>(t) * p.kv_tok + static_cast<int64_t>(g) * p.kv_head + c8 * 16;
+        rk[u] = ld_nc_v4(p.k8 + off);
+        rv[u] = ld_nc_v4(p.v8 + off);
+        sk[u] = p.ksc[static_cast<int64_t>(t) * p.Hkv + g];
+        sv[u] = p.vsc[static_cast<int64_t>(t) * p.Hkv + g];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < ROWS; ++u) {
+      const int64_t row = r0 + u * stride;
+      if (row >= rows) continue;
+      const int t = static_cast<int>(row / p.Hkv), g = static_cast<int>(row % p.Hkv);
+      if (c8 == 0) p.kcol[static_cast<int64_t>(g) * p.Lp + t] = (t < p.L) ? sk[u] * p.scale_log2 : 0.f;
+      if (t >= p.L) continue;
+      const uint32_t wk[4] = {rk[u].x, rk[u].y, rk[u].z, rk[u].w};
+      const uint32_t wv[4] = {rv[u].x, rv[u].y, rv[u].z, rv[u].w};
+      const uint32_t s2 = pack_f16x2(sv[u], sv[u]);
+      uint32_t fk[8], fv[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        fk[2 * q] = e4m3x2_to_f16x2(wk[q]);
+        fk[2 * q + 1] = e4m3x2_to_f16x2(wk[q] >> 16);
+        fv[2 * q] = hmul2_u32(e4m3x2_to_f16x2(wv[q]), s2);
+        fv[2 * q + 1] = hmul2_u32(e4m3x2_to_f16x2(wv[q] >> 16), s2);
+      }
+      const int64_t o = (static_cast<int64_t>(t) * p.Hkv + g) * 128 + c8 * 16;
+      uint4* dk = reinterpret_cast<uint4*>(p.kf + o);
+      uint4* dv = reinterpret_cast<uint4*>(p.vf + o);
+      dk[0] = make_uint4(fk[0], fk[1], fk[2], fk[3]);
+      dk[1] = make_uint4(fk[4], fk[5], fk[6], fk[7]);
+      dv[0] = make_uint4(fv[0], fv[1], fv[2], fv[3]);
+      dv[1] = make_uint4(fv[4], fv[5], fv[6], fv[7]);
+    }
+  }
+}
+
+}  // namespace hs2
