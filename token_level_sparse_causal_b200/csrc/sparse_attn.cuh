@@ -8,7 +8,7 @@
 // windows cover, loaded as whole tiles by TMA, with the band mask
 // i - W < j <= i.
 //
-// The arithmetic per work item is that of flash_fwd_kernel<FLASH_SPARSE>: an
+// The per-tile arithmetic is that of kernel (1) (flash_fwd_kernel): an
 // item is (query block b, KV head g, pair of 128-row M tiles), each M tile
 // 128/G tokens x G heads of the block sharing the block's list, whose K/V rows
 // are gathered with 16-byte cp.async into 128-byte-swizzled shared memory
@@ -29,10 +29,12 @@
 //   * the first P V of an item waits only for the previous epilogue of the
 //     same M tile to have read O (o_free); its S products do not wait.
 //
-// Roles (12 warps), as in flash_fwd_kernel: warp 0 loads Q by TMA, warp 1
-// issues every MMA, warps 2-3 load lists and gather K/V (with an FP8 cache:
-// also convert Q and the K/V codes to f16), warps 4-7 / 8-11 run the softmax
-// and epilogue of M tile A / B.  Every wait is bounded; a wait that runs out
+// Roles (12 warps), as in flash_fwd_kernel: warp 1 issues every MMA, warps
+// 4-7 / 8-11 run the softmax and epilogue of M tile A / B; with a bf16 cache
+// warps 0, 2 and 3 load the lists, gather K/V and (one thread) load Q; with an
+// FP8 cache warp 0 loads Q by TMA and warps 2-3 convert it and gather and
+// convert the K/V codes to f16; in window mode warp 0 loads Q and whole K/V
+// tiles by TMA.  Every wait is bounded; a wait that runs out
 // records HS2_ERR_TIMEOUT and the CTA winds down.
 #pragma once
 
