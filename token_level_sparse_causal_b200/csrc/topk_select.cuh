@@ -228,6 +228,71 @@ __device__ void bitonic_sort_smem(uint32_t* a, int np) {
   }
 }
 
+// One streaming pass over a row: appends the raw bits and the position of
+// every value whose order key is >= tau to (ckey, cpos) (at most SEL_CAP are
+// stored; *count receives the total).  FAST: tau is the key of a positive
+// float, and for any fp32 v, order_key(v) >= tau exactly when the bits of v
+// as a signed integer are >= those of that float (negative values, -0.0 and
+// negative NaNs are negative integers; positive NaNs lie above +inf in both
+// orders), so one integer compare decides.  Each thread first counts its
+// values (16 in flight), the warp forms a prefix with one shared atomic, and
+// only then do lanes with hits store them.
+template <bool FAST>
+__device__ __forceinline__ void gather_pass(const float4* row4, int n4, uint32_t tau, uint32_t* ckey,
+                                            uint32_t* cpos, uint32_t* count) {
+  constexpr int U = 4;  // float4 loads in flight per thread
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int tau_i = static_cast<int>(tau & 0x7FFFFFFFu);
+  auto hit = [&](float f, bool live) -> bool {
+    return FAST ? (__float_as_int(f) >= tau_i) : (live && order_key(f) >= tau);
+  };
+#pragma unroll 1
+  for (int base4 = 0; base4 < n4; base4 += SEL_THREADS * U) {
+    float4 v[U];
+    bool live[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i4 = base4 + u * SEL_THREADS + tid;
+      live[u] = i4 < n4;
+      // -inf pads the tail: a negative integer, never >= a positive float
+      v[u] = live[u] ? __ldg(row4 + i4) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
+    uint32_t c = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      c += (hit(v[u].x, live[u]) ? 1u : 0u) + (hit(v[u].y, live[u]) ? 1u : 0u) + (hit(v[u].z, live[u]) ? 1u : 0u) +
+           (hit(v[u].w, live[u]) ? 1u : 0u);
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t wtot = __shfl_sync(0xffffffffu, incl, 31);
+    if (wtot == 0) continue;  // warp-uniform
+    uint32_t wbase = 0;
+    if (lane == 31) wbase = atomicAdd(count, wtot);
+    uint32_t at = __shfl_sync(0xffffffffu, wbase, 31) + incl - c;
+    if (c) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t p0 = static_cast<uint32_t>(base4 + u * SEL_THREADS + tid) * 4u;
+        const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (hit(vv[e], live[u])) {
+            if (at < SEL_CAP) {
+              ckey[at] = __float_as_uint(vv[e]);
+              cpos[at] = p0 + e;
+            }
+            ++at;
+          }
+        }
+      }
+    }
+  }
+}
+
 // Shared memory of topk_select_kernel (dynamic).
 struct SelSmem {
   uint32_t ckey[SEL_CAP];    // gathered candidates: order keys ...
@@ -240,7 +305,8 @@ struct SelSmem {
 };
 
 // Kernel (3).  For rows with n > k candidates, the fast path reads the row
-// once: a strided sample of SEL_SAMPLES values gives a threshold tau (the
+// once: a sample of up to SEL_SAMPLES values (groups of 8 consecutive values
+// spread evenly over the row) gives a threshold tau (the
 // sample's q-th largest, q chosen so that about 2k values are expected at
 // or above it; tau = 0 when the whole row fits in shared memory), every
 // value >= tau is gathered into shared memory, and there the k-th largest T
@@ -270,80 +336,41 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const SelPa
     const int n4 = n_c >> 2;  // n_c is a multiple of 64
     const uint32_t k = static_cast<uint32_t>(p.topk);
 
-    // ---- threshold from a strided sample
+    // ---- threshold from a sample of whole 32-byte sectors: groups of 8
+    // consecutive values spread evenly over the row (a scattered sample
+    // would touch a separate DRAM burst per value)
     uint32_t tau = 0;
     if (n_c > SEL_CAP) {
-      // one sample per 8 values, 1024 .. SEL_SAMPLES of them
-      // about one sample per 8 values: 1024, 2048 or 4096 of them
+      // 1024, 2048 or 4096 sampled values (128, 256 or 512 groups)
       const int lg = n_c >= 8 * SEL_SAMPLES ? 12 : n_c >= 8 * 2048 ? 11 : 10;
       const int ns = 1 << lg;
-      float sv[SEL_SAMPLES / SEL_THREADS];  // every load in flight at once
-#pragma unroll
-      for (int u = 0; u < SEL_SAMPLES / SEL_THREADS; ++u) {
-        const int i = tid + u * SEL_THREADS;
-        const int j = static_cast<int>((static_cast<int64_t>(i) * n_c) >> lg) + ((n_c >> lg) >> 1);
-        sv[u] = (i < ns) ? __ldg(row + j) : 0.f;
+      if (tid < (ns >> 3)) {  // group tid starts at a multiple of 8, ends before n_c
+        const int j0 = static_cast<int>((static_cast<int64_t>(tid) * n_c) >> (lg - 3)) & ~7;
+        const float4 a = __ldg(row4 + (j0 >> 2)), c = __ldg(row4 + (j0 >> 2) + 1);
+        uint4 o0 = make_uint4(order_key(a.x), order_key(a.y), order_key(a.z), order_key(a.w));
+        uint4 o1 = make_uint4(order_key(c.x), order_key(c.y), order_key(c.z), order_key(c.w));
+        *reinterpret_cast<uint4*>(S.samp + 8 * tid) = o0;
+        *reinterpret_cast<uint4*>(S.samp + 8 * tid + 4) = o1;
       }
-#pragma unroll
-      for (int u = 0; u < SEL_SAMPLES / SEL_THREADS; ++u)
-        if (tid + u * SEL_THREADS < ns) S.samp[tid + u * SEL_THREADS] = order_key(sv[u]);
       __syncthreads();
       const int64_t qq = (2 * static_cast<int64_t>(k) * ns + n_c - 1) / n_c;
       const uint32_t q = static_cast<uint32_t>(qq < 1 ? 1 : (qq > ns ? ns : qq));
       uint32_t unused;
       tau = smem_kth_largest(S.samp, ns, q, S.hist, S.warp_sums, S.sh, &unused);
     }
-    // ---- gather every value >= tau (warp-aggregated appends; order is
-    // restored by the sort below)
+    // ---- gather every value >= tau: the raw fp32 bits and positions go to
+    // shared memory (warp-aggregated appends; order is restored below), then
+    // the bits are mapped to order keys
     if (tid == 0) S.count = 0;
     __syncthreads();
-    constexpr int U = 4;  // float4 loads in flight per thread
-#pragma unroll 1
-    for (int base4 = 0; base4 < n4; base4 += SEL_THREADS * U) {
-      float4 v[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i4 = base4 + u * SEL_THREADS + tid;
-        v[u] = (i4 < n4) ? __ldg(row4 + i4) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-      }
-      uint32_t mask = 0;  // bit 4u + e: value e of load u is >= tau
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i4 = base4 + u * SEL_THREADS + tid;
-        const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          mask |= ((i4 < n4) && order_key(vv[e]) >= tau ? 1u : 0u) << (4 * u + e);
-      }
-      // warp prefix of the counts, one shared atomic per warp
-      const uint32_t c = static_cast<uint32_t>(__popc(mask));
-      uint32_t incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const uint32_t wtot = __shfl_sync(0xffffffffu, incl, 31);
-      uint32_t wbase = 0;
-      if (lane == 31 && wtot) wbase = atomicAdd(&S.count, wtot);
-      uint32_t at = __shfl_sync(0xffffffffu, wbase, 31) + incl - c;
-      if (mask) {
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int i4 = base4 + u * SEL_THREADS + tid;
-          const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (mask & (1u << (4 * u + e))) {
-              if (at < SEL_CAP) {
-                S.ckey[at] = order_key(vv[e]);
-                S.cpos[at] = static_cast<uint32_t>(i4 * 4 + e);
-              }
-              ++at;
-            }
-          }
-        }
-      }
+    if (tau > 0x80000000u)
+      gather_pass<true>(row4, n4, tau, S.ckey, S.cpos, &S.count);
+    else
+      gather_pass<false>(row4, n4, tau, S.ckey, S.cpos, &S.count);
+    __syncthreads();
+    {
+      const int ng = static_cast<int>(min(S.count, static_cast<uint32_t>(SEL_CAP)));
+      for (int i = tid; i < ng; i += SEL_THREADS) S.ckey[i] = order_key(__uint_as_float(S.ckey[i]));
     }
     __syncthreads();
     const uint32_t cnt_g = S.count;
