@@ -278,10 +278,11 @@ def cpu_baseline(wl, x, seconds_target: float) -> dict:
 
 # ------------------------------------------------------------- cuda arm --
 
-def select_alone(hs2, torch, shape, q0, k, ks, out, dev, timed, nblk=64):
+def select_alone(hs2, torch, shape, q0, k, ks, out, dev, timed, nblk=256):
     """Kernel (3) by itself on the importance rows of the last `nblk` query
-    blocks (the longest rows; a strip larger than L2, so it streams from
-    HBM): device time and the row bytes it must read."""
+    blocks (the longest rows; at 128k a 1.07 GB strip of 2048 rows, larger
+    than L2 and several waves of resident CTAs, so it streams from HBM):
+    device time and the row bytes it must read."""
     nb = shape.L // shape.block
     b0 = max(0, nb - nblk)
     n_c = lambda b: max(0, min(shape.L, shape.block * (b + 1)) - shape.recent)
@@ -540,6 +541,44 @@ def run_reference(args, wl, rank, world):
             "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_stage(args, wl):
+    """One stage alone on a reduced-footprint copy of the workload (same L and
+    input recipe, the heads given by --heads, no sparse layers) -- the case
+    an ncu capture of that stage's kernel runs on.  select: kernel (1) for
+    the LSE, then kernel (3) alone on the strip of the longest rows."""
+    import torch
+    from token_level_sparse_causal_b200 import build, hs2, inputs
+
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hq, hkv = (int(t) for t in args.heads.split("/")) if args.heads else (wl.Hq, wl.Hkv)
+    my = wl.scaled(name=f"{wl.name}_stage_h{hq}x{hkv}", Hq=hq, Hkv=hkv, n_sparse=0)
+    x = inputs.make_inputs(my, device=dev, with_needles=bool(my.needles))
+    q0, k, v = x["q_layers"][0], x["k"], x["v"]
+    ks, vs = x.get("k_scale"), x.get("v_scale")
+    fp8_cache = k.dtype == torch.uint8
+    shape = hs2.make_shape(q0, k, my.topk, my.recent, kv_dtype=hs2.HS2_KV_E4M3 if fp8_cache else hs2.HS2_KV_BF16)
+    out = hs2.alloc_outputs(shape, q0)
+    stream = torch.cuda.current_stream()
+    hs2.hs2_attn_fwd(shape, q0, k, v, ks, vs, out["o"], out["lse"], stream)
+
+    def timed(fn, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    res = select_alone(hs2, torch, shape, q0, k, ks, out, dev, timed)
+    hs2.hs2_sync(stream)
+    return {"stage": "select_alone", "workload": my.name, "L": my.L, "Hq": hq, "Hkv": hkv, **res}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -550,12 +589,17 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample size for cpu_baseline")
+    ap.add_argument("--stage", choices=["select"], help="time one stage alone (1 GPU) and print its line")
+    ap.add_argument("--heads", help="with --stage: query/KV heads of the reduced copy, e.g. 16/8")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "cuda":
         ap.error("--warmup must be >= 3")
 
     from token_level_sparse_causal_b200 import inputs
     wl = inputs.WORKLOADS[args.workload]
+    if args.stage:
+        print(json.dumps(run_stage(args, wl)), flush=True)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     dist = None
