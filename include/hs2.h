@@ -88,8 +88,10 @@ typedef struct hs2_shape {
  *
  * workspace / workspace_bytes: scratch device memory for importance strips.
  *   workspace == NULL: *workspace_bytes receives the recommended size (whole
- *   path in as few strips as possible, capped so a strip stays L2-resident)
- *   and nothing else happens.  Otherwise *workspace_bytes is the size of
+ *   path in as few strips as possible, capped at 64 MiB so a strip stays
+ *   L2-resident, but never below 296 of the longest rows, two per SM, so that
+ *   a select launch over long rows keeps the GPU busy) and nothing else
+ *   happens.  Otherwise *workspace_bytes is the size of
  *   `workspace` (16-byte aligned); it must be at least
  *   Hkv * roundup(L - recent, 64) * 4 bytes (one block per strip), else
  *   HS2_ERR_WORKSPACE.  The workspace holds no state between calls.
@@ -169,6 +171,19 @@ int hs2_sync(void* stream);
 /* Full causal attention forward with LSE only (kernel 1 of the path). */
 int hs2_attn_fwd(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
                  const float* v_scale, void* o, float* lse, void* stream);
+
+/*
+ * hs2_attn_fwd as hs2_full_attn_select runs it: with an e4m3 cache and a
+ * workspace of at least the size this call reports (workspace == NULL: the
+ * size goes to *workspace_bytes, nothing else happens; 0 for a bf16 cache),
+ * the cache is first converted once into the workspace (an f16 copy of K and
+ * V plus the K column scales) and kernel (1) loads f16 tiles from it;
+ * otherwise this is hs2_attn_fwd.  Results are identical to hs2_attn_fwd.
+ * workspace: 16-byte aligned; no state is kept between calls.
+ */
+int hs2_attn_fwd_ws(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
+                    const float* v_scale, void* o, float* lse, void* workspace, size_t* workspace_bytes,
+                    void* stream);
 
 /*
  * Importance rows (kernel 2) for query blocks [b0, b1), given the full

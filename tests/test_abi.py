@@ -67,9 +67,27 @@ def test_workspace_query_is_host_only(lib):
     s = _shape(L=131072, Hq=64, Hkv=8, q_tok_stride=64 * 128, kv_tok_stride=8 * 128)
     n = hs2.workspace_bytes(s)
     min_ws = 8 * (131072 - 128) * 4
-    assert min_ws <= n <= max(min_ws, 64 << 20)
+    row = (131072 - 128) * 4  # the longest importance row
+    # strips fit L2 (64 MiB) or, for long rows, hold at least 296 rows (two per SM)
+    assert min_ws <= n <= max(min_ws, 64 << 20, 296 * row + 4096)
+    assert n >= min(296 * row, 64 << 20)
     small = _shape(L=1024)
     assert hs2.workspace_bytes(small) >= 2 * (1024 - 128) * 4
+
+
+def test_fp8_workspaces_hold_the_layer_copy(lib):
+    """With an e4m3 cache the recommended full-layer workspace, and the one
+    hs2_attn_fwd_ws asks for, hold the f16 copy of K and V plus the K column
+    scales; a bf16 cache needs none for kernel (1)."""
+    L, Hkv = 131072, 8
+    copy = 2 * L * Hkv * 128 * 2 + Hkv * L * 4
+    s8 = _shape(L=L, Hq=64, Hkv=Hkv, q_tok_stride=64 * 128, kv_tok_stride=Hkv * 128, kv_dtype=hs2.HS2_KV_E4M3)
+    assert hs2.workspace_bytes(s8) >= Hkv * (L - 128) * 4 + copy
+    assert copy <= hs2.attn_fwd_workspace_bytes(s8) <= copy + 1024
+    s16 = _shape(L=L, Hq=64, Hkv=Hkv, q_tok_stride=64 * 128, kv_tok_stride=Hkv * 128)
+    assert hs2.attn_fwd_workspace_bytes(s16) == 0
+    assert lib.hs2_attn_fwd_ws(ctypes.byref(s8), None, None, None, None, None, None, None, None, None,
+                               None) == hs2.HS2_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("kw,code", [

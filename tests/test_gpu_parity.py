@@ -474,6 +474,12 @@ def test_fp8_layer_copy_equals_in_kernel_conversion(L, Hq, Hkv):
     hs2.hs2_attn_fwd(shape, q0, k, v, ks, vs, o1, lse1)
     hs2.hs2_sync()
     assert torch.equal(o1, outs[1][0]) and torch.equal(lse1, outs[1][1])
+    # kernel (1) alone through the layer copy (hs2_attn_fwd_ws)
+    ws1 = torch.empty(hs2.attn_fwd_workspace_bytes(shape) // 4 + 4, device=DEV, dtype=torch.float32)
+    o2, lse2 = torch.empty_like(q0), torch.empty((Hq, L), device=DEV, dtype=torch.float32)
+    hs2.hs2_attn_fwd_ws(shape, q0, k, v, ks, vs, o2, lse2, ws1)
+    hs2.hs2_sync()
+    assert torch.equal(o2, o1) and torch.equal(lse2, lse1)
 
 
 # -------------------------------------------------- device-side failures --

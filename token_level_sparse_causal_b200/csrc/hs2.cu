@@ -498,13 +498,21 @@ size_t min_workspace(const hs2_shape* s) {
 
 constexpr size_t kStripCap = size_t(64) << 20;  // keep one strip L2-resident
 
-// Strips in as few launches as the L2 cap allows; with an e4m3 cache, plus
-// room for the layer's f16 copy (dequant_bytes).
+// Rows a select launch should have at least: two per SM of a B200 (148 SMs),
+// so that the per-row latency of long rows is overlapped across the GPU.
+constexpr size_t kSelectRows = 296;
+
+// Strips in as few launches as the L2 cap allows, but never fewer rows per
+// strip than kSelectRows (long rows then stream from HBM instead of L2:
+// cheaper than launches of a few latency-bound rows); with an e4m3 cache,
+// plus room for the layer's f16 copy (dequant_bytes).
 size_t recommended_workspace(const hs2_shape* s) {
   size_t whole = 0;
   const int nb = s->L / 64;
   for (int b = 0; b < nb; ++b) whole += static_cast<size_t>(s->Hkv) * strip_stride(s, b) * 4u;
-  const size_t strips = std::max(min_workspace(s), std::min(whole, kStripCap));
+  const size_t row_bytes = static_cast<size_t>(strip_stride(s, nb - 1)) * 4u;
+  const size_t cap = std::max(kStripCap, kSelectRows * row_bytes);
+  const size_t strips = std::max(min_workspace(s), std::min(whole, cap));
   return strips + (s->kv_dtype == HS2_KV_E4M3 ? dequant_bytes(s) : 0u);
 }
 
@@ -579,6 +587,29 @@ int hs2_attn_fwd(const hs2_shape* shape, const void* q, const void* k, const voi
   if (!q || !o || !lse) return HS2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || !aligned16(lse)) return HS2_ERR_UNSUPPORTED;
   return launch_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, static_cast<cudaStream_t>(stream));
+}
+
+int hs2_attn_fwd_ws(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
+                    const float* v_scale, void* o, float* lse, void* workspace, size_t* workspace_bytes,
+                    void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!workspace_bytes) return HS2_ERR_INVALID_ARG;
+  const bool kv8 = shape->kv_dtype == HS2_KV_E4M3;
+  if (!workspace) {
+    *workspace_bytes = kv8 ? dequant_bytes(shape) : 0u;
+    return HS2_OK;
+  }
+  if ((rc = check_kv(shape, k, v, k_scale, v_scale))) return rc;
+  if (!q || !o || !lse) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || !aligned16(workspace)) return HS2_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (kv8 && *workspace_bytes >= dequant_bytes(shape)) {
+    const DequantBuf dqb = dequant_carve(shape, static_cast<uint8_t*>(workspace));
+    if ((rc = launch_dequant(shape, k, v, k_scale, v_scale, dqb, st))) return rc;
+    return launch_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, st, &dqb);
+  }
+  return launch_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, st);
 }
 
 int hs2_swa_attn(const hs2_shape* shape, const void* q, const void* k, const void* v, int32_t window, void* o,

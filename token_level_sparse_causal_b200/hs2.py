@@ -23,7 +23,7 @@ EXPORTS = ("hs2_full_attn_select", "hs2_sparse_attn", "hs2_sync", "hs2_attn_fwd"
            "hs2_topk_select", "hs2_strerror", "hs2_debug_set", "hs2_version", "hs2_launch_count",
            "hs2_full_attn_select_static", "hs2_exp2_check", "hs2_quantize_kv", "hs2_block_select",
            "hs2_full_attn_select_blocks", "hs2_swa_attn", "hs2_sparse_decode",
-           "hs2_sparse_decode_workspace")
+           "hs2_sparse_decode_workspace", "hs2_attn_fwd_ws")
 
 
 class Hs2Shape(ctypes.Structure):
@@ -52,6 +52,8 @@ _SIGS = {
     "hs2_sparse_attn": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "hs2_sync": [_vp],
     "hs2_attn_fwd": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "hs2_attn_fwd_ws": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                        ctypes.POINTER(ctypes.c_size_t), _vp],
     "hs2_swa_attn": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _i32, _vp, _vp, _vp],
     "hs2_sparse_decode": [ctypes.POINTER(Hs2Shape), _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                           ctypes.c_size_t, _vp],
@@ -154,6 +156,25 @@ def hs2_sparse_attn(shape, q, k, v, k_scale, v_scale, idx, cnt, o, stream=None) 
 def hs2_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, stream=None) -> None:
     _check(lib().hs2_attn_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale),
                               _ptr(o), _ptr(lse), _stream(stream)), "hs2_attn_fwd")
+
+
+def attn_fwd_workspace_bytes(shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().hs2_attn_fwd_ws(ctypes.byref(shape), None, None, None, None, None, None, None, None,
+                                 ctypes.byref(n), None), "hs2_attn_fwd_ws(size query)")
+    return int(n.value)
+
+
+def hs2_attn_fwd_ws(shape, q, k, v, k_scale, v_scale, o, lse, workspace, stream=None) -> None:
+    """Kernel (1) as the full layer runs it.  A null workspace pointer is the
+    C call's size query, so without a workspace this is hs2_attn_fwd."""
+    if workspace is None or workspace.numel() == 0:
+        hs2_attn_fwd(shape, q, k, v, k_scale, v_scale, o, lse, stream)
+        return
+    n = ctypes.c_size_t(workspace.numel() * workspace.element_size())
+    _check(lib().hs2_attn_fwd_ws(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale),
+                                 _ptr(o), _ptr(lse), _ptr(workspace), ctypes.byref(n), _stream(stream)),
+           "hs2_attn_fwd_ws")
 
 
 def sparse_decode_workspace_bytes(shape, n: int) -> int:
