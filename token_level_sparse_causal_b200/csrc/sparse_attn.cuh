@@ -435,6 +435,18 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           for (int j = 0; j < w.nt && ok; ++j) {
             const int u = u0 + j;
             const int s = u % FL_STAGES;
+            // the next tile's rows start moving into L2 now: its gather can
+            // only begin once a stage frees, and rows missing L2 would
+            // otherwise set that gather's length
+            if (j + 1 < w.nt) {  // 4 lines of 128 B per listed position (K and V rows)
+              for (int q = pt; q < 4 * 128; q += NLD) {
+                const int pj = pos_s[(j + 1) * 128 + (q >> 2)];
+                if (pj >= 0) {
+                  const int64_t off = static_cast<int64_t>(pj) * p.kv_tok - chunk * 8 + (q & 1) * 64;
+                  prefetch_l2(((q & 2) ? vg : kg) + off);
+                }
+              }
+            }
             if (u >= FL_STAGES &&
                 !mbar_wait(&bars->empty[s], ((u / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 325)) {
               ok = false;
