@@ -163,13 +163,15 @@ __device__ void select_radix_global(const float4* row4, int n4, uint32_t k, uint
 // k-th largest of n keys in shared memory, by radix select (digits of 11, 11
 // and 10 bits, histogram in `hist`): returns T and sets *krem to the number
 // of keys equal to T among the k largest.  Requires 1 <= k <= n.  Every
-// thread gets the same result.
+// thread gets the same result.  passes = 2 stops after the top 22 bits and
+// returns the lower edge of the bin holding the k-th largest (a lower bound
+// within 2^10 key steps; *krem is then meaningless).
 __device__ uint32_t smem_kth_largest(const uint32_t* keys, int n, uint32_t k, uint32_t* hist, uint32_t* warp_sums,
-                                     uint32_t* sh, uint32_t* krem_out) {
+                                     uint32_t* sh, uint32_t* krem_out, int passes = 3) {
   const int tid = threadIdx.x;
   uint32_t prefix = 0, pmask = 0, krem = k;
 #pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
+  for (int pass = 0; pass < passes; ++pass) {
     const int shift = (pass == 0) ? 21 : (pass == 1) ? 10 : 0;
     const int nbins = (pass == 2) ? 1024 : 2048;
     for (int i = tid; i < nbins; i += SEL_THREADS) hist[i] = 0;
@@ -355,8 +357,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const SelPa
       __syncthreads();
       const int64_t qq = (2 * static_cast<int64_t>(k) * ns + n_c - 1) / n_c;
       const uint32_t q = static_cast<uint32_t>(qq < 1 ? 1 : (qq > ns ? ns : qq));
-      uint32_t unused;
-      tau = smem_kth_largest(S.samp, ns, q, S.hist, S.warp_sums, S.sh, &unused);
+      uint32_t unused;  // a lower bound of the sample's q-th largest is enough for tau
+      tau = smem_kth_largest(S.samp, ns, q, S.hist, S.warp_sums, S.sh, &unused, 2);
     }
     // ---- gather every value >= tau: the raw fp32 bits and positions go to
     // shared memory (warp-aggregated appends; order is restored below), then
