@@ -134,14 +134,18 @@ def _crafted_rows(n, rng):
         np.where(rng.random(n) < 0.5, -0.0, 0.0).astype(np.float32),        # +-0 only
         np.exp(-rng.random(n) * 80).astype(np.float32),                     # wide dynamic range
         np.concatenate([np.zeros(n - 1100, np.float32), np.full(1100, 1e-3, np.float32)]),  # tail-heavy
+        rng.standard_normal(n).astype(np.float32),                          # signed: a positive threshold
+        # with negative values, -0.0 and huge magnitudes beneath it
+        np.where(rng.random(n) < 0.1, -3.0e38, rng.standard_normal(n) * 1e-20).astype(np.float32),
+        -rng.random(n).astype(np.float32) - 1.0,                            # all negative
     ]
     return kinds
 
 
 def test_select_crafted_rows_bit_exact():
-    L, Hkv, topk, recent = 8192, 6, 1024, 128
-    shape = hs2.Hs2Shape(L=L, Hq=12, Hkv=Hkv, d=128, block=64, topk=topk, recent=recent, kv_dtype=0,
-                         q_tok_stride=12 * 128, q_head_stride=128, kv_tok_stride=Hkv * 128, kv_head_stride=128)
+    L, Hkv, topk, recent = 8192, 9, 1024, 128
+    shape = hs2.Hs2Shape(L=L, Hq=18, Hkv=Hkv, d=128, block=64, topk=topk, recent=recent, kv_dtype=0,
+                         q_tok_stride=18 * 128, q_head_stride=128, kv_tok_stride=Hkv * 128, kv_head_stride=128)
     nb = L // 64
     rng = np.random.default_rng(5)
     for b0, b1 in [(0, 24), (100, 104), (nb - 3, nb)]:
@@ -169,10 +173,20 @@ def test_select_crafted_rows_bit_exact():
         assert np.all(idx_h[:, untouched] == -9) and np.all(cnt_h[:, untouched] == -9)
 
 
+def _threshold_sample_positions(n_c):
+    """Where kernel (3)'s threshold sample reads a row of n_c > 4096
+    candidates: 2^(lg-3) groups of 8 consecutive values, group t starting at
+    (t * n_c >> (lg - 3)) rounded down to a multiple of 8."""
+    lg = 12 if n_c >= 8 * 4096 else 11 if n_c >= 8 * 2048 else 10
+    ng = 1 << (lg - 3)
+    j0 = ((np.arange(ng, dtype=np.int64) * n_c) >> (lg - 3)) & ~7
+    return (j0[:, None] + np.arange(8)[None, :]).ravel()
+
+
 def test_select_rows_that_defeat_the_sample_bit_exact():
     """Long rows (n > 8192) where the single-read path must give up: all
     values equal (too many gathered), and a row whose large values sit exactly
-    where a strided sample of 4096 looks, so the sample overestimates the
+    where the threshold sample looks, so the sample overestimates the
     threshold (too few gathered).  The exact radix path then decides, and the
     lists must still equal the oracle's."""
     L, Hkv, topk, recent = 16384, 3, 1024, 128
@@ -185,8 +199,7 @@ def test_select_rows_that_defeat_the_sample_bit_exact():
     rows = np.full((Hkv, b1 - b0, stride), np.nan, np.float32)
     for bi, b in enumerate(range(b0, b1)):
         n_c = orc.n_candidates(64 * (b + 1), recent)
-        S = 4096
-        sample_pos = (np.arange(S, dtype=np.int64) * n_c) // S + (n_c // S) // 2
+        sample_pos = _threshold_sample_positions(n_c)
         trap = (rng.random(n_c) * 1e-3).astype(np.float32)
         trap[sample_pos[:500]] = 1.0          # 500 large values, all of them sampled
         rows[0, bi, :n_c] = np.full(n_c, 0.25, np.float32)
