@@ -320,7 +320,33 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           ok = false;
           break;
         }
-        if (q_thread && w.nt > 0) {  // bf16: Q of the item, once the previous item's S products ran
+        // entries past the count, and entries outside [0, e_b) (reported),
+        // become -1: never read, always masked
+        const int32_t* list = p.idx + (static_cast<int64_t>(w.g) * p.nb + w.b) * p.list_len;
+        constexpr int LB = 6;  // list loads in flight per thread (a 1152-entry list: 2 or 3 rounds)
+        for (int i0 = pt; i0 < w.nt * 128; i0 += LB * NLD) {
+          int e[LB];
+#pragma unroll
+          for (int v = 0; v < LB; ++v) {
+            const int i = i0 + v * NLD;
+            e[v] = (i < w.cnt) ? __ldg(list + i) : -1;
+          }
+#pragma unroll
+          for (int v = 0; v < LB; ++v) {
+            const int i = i0 + v * NLD;
+            if (i < w.nt * 128) {
+              if (i < w.cnt && (e[v] < 0 || e[v] >= w.e_b)) {
+                report(HS2_ERR_INDEX, 328);
+                e[v] = -1;
+              }
+              pos_s[i] = e[v];
+            }
+          }
+        }
+        mbar_arrive(&bars->list_full[buf]);
+        // bf16: Q of the item, once the previous item's S products ran (after
+        // this thread's share of the list, so the list is not held up)
+        if (q_thread && w.nt > 0) {
           if (loaded > 0 && !mbar_wait(&bars->q_empty, (loaded - 1) & 1, p.limit_ns, abort_flag, 301)) {
             ok = false;
             break;
@@ -335,21 +361,6 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           }
           ++loaded;
         }
-        // entries past the count, and entries outside [0, e_b) (reported),
-        // become -1: never read, always masked
-        const int32_t* list = p.idx + (static_cast<int64_t>(w.g) * p.nb + w.b) * p.list_len;
-        for (int i = pt; i < w.nt * 128; i += NLD) {
-          int e = -1;
-          if (i < w.cnt) {
-            e = __ldg(list + i);
-            if (e < 0 || e >= w.e_b) {
-              report(HS2_ERR_INDEX, 328);
-              e = -1;
-            }
-          }
-          pos_s[i] = e;
-        }
-        mbar_arrive(&bars->list_full[buf]);
         // the loaders read each other's entries too: wait for all of them (bounded)
         if (!mbar_wait(&bars->list_full[buf], (ii >> 1) & 1, p.limit_ns, abort_flag, 327)) {
           ok = false;
