@@ -101,6 +101,21 @@ def recorded_traffic(workload: str, profile=FA_TRAFFIC_PROFILE):
         return None
 
 
+def data_recipe(wl) -> str:
+    """One line naming the synthetic input recipe of a workload."""
+    k = "K from a 64-component Gaussian mixture, std 0.3" if wl.k_dist == "gmm64" else "Q/K/V ~ N(0,1)"
+    n = wl.needles
+    if n and n[0] == "total":
+        k += f", {n[1]} planted needle keys"
+    elif n and n[0] == "per_kv_head":
+        k += f", {n[1]} planted needle keys per KV head"
+    elif n and n[0] == "chains":
+        k += f", {n[1]} multi-hop needle chains of {n[2]} keys"
+    if wl.kv_dtype == "e4m3":
+        k += ", K/V as e4m3 codes + per-token fp32 scale"
+    return f"synthetic (seeded {wl.seed}; {k})"
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -477,7 +492,7 @@ def run_cuda(args, wl, rank, world, dist):
         "p50_ms": float(np.percentile(per, 50)), "p99_ms": float(np.percentile(per, 99)),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 Q, e4m3 K/V (f16 MMA)" if fp8_cache else "bf16",
-        "data": "synthetic (seeded; K from a 64-component Gaussian mixture, std 0.3)",
+        "data": data_recipe(wl),
         "config": {"workload": wl.name, "L": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
                    "layers": f"1 full + {wl.n_sparse} sparse", "topk": wl.topk, "recent": wl.recent,
                    "block": wl.block, "batch_per_gpu": 1, "parallelism": f"independent sequence per GPU x{world}",
