@@ -1,0 +1,45 @@
+"""Host-side pieces of bench.py that decide what its JSON line claims: the
+committed kernel (1) DRAM traffic is reported only for the workload and the
+kernel sources it was captured on, and each workload's line names its own
+input recipe."""
+import os
+
+import bench
+from token_level_sparse_causal_b200 import inputs
+
+
+def test_recorded_traffic_only_for_its_own_workload_and_sources(tmp_path):
+    good = tmp_path / "dram.md"
+    good.write_text("# capture\n\n"
+                    "- workload: c3_L131072_h64x8_gmm\n"
+                    "- dram_bytes_per_launch: 12345\n"
+                    f"- kernel_source_sha256_16: {bench.kernel_source_hash()}\n")
+    assert bench.recorded_traffic("c3_L131072_h64x8_gmm", str(good)) == 12345.0
+    assert bench.recorded_traffic("c4_L262144_h64x8_chains", str(good)) is None
+    stale = tmp_path / "stale.md"
+    stale.write_text("- workload: c3_L131072_h64x8_gmm\n- dram_bytes_per_launch: 12345\n"
+                     "- kernel_source_sha256_16: 0000000000000000\n")
+    assert bench.recorded_traffic("c3_L131072_h64x8_gmm", str(stale)) is None
+    assert bench.recorded_traffic("c3_L131072_h64x8_gmm", str(tmp_path / "missing.md")) is None
+
+
+def test_committed_traffic_summary_is_well_formed():
+    """The committed summary names its workload and a per-launch byte count
+    (whether its hash is current depends on the kernel sources)."""
+    fields = {}
+    for line in open(bench.FA_TRAFFIC_PROFILE):
+        if line.strip().startswith("- ") and ":" in line:
+            k, v = line.strip()[2:].split(":", 1)
+            fields[k.strip()] = v.strip()
+    assert fields["workload"] == inputs.WORKLOADS["c3"].name
+    assert int(fields["dram_bytes_per_launch"]) == int(fields["dram_read_bytes"]) + int(fields["dram_write_bytes"])
+
+
+def test_data_recipe_names_each_workloads_inputs():
+    r = {k: bench.data_recipe(w) for k, w in inputs.WORKLOADS.items()}
+    assert "Gaussian mixture" in r["c3"] and "needle" not in r["c3"]
+    assert "16 planted needle keys" in r["c1"]
+    assert "256 planted needle keys per KV head" in r["c2"]
+    assert "8 multi-hop needle chains of 4 keys" in r["c4"]
+    assert "e4m3" in r["c5"] and "1024 planted needle keys per KV head" in r["c5"]
+    assert all(v.startswith("synthetic (seeded ") for v in r.values())
