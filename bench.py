@@ -101,6 +101,15 @@ def recorded_traffic(workload: str, profile=FA_TRAFFIC_PROFILE):
         return None
 
 
+def arm_config(wl, world: int) -> dict:
+    """The `config` object of both arms' JSON lines (the same workload)."""
+    q_gb = wl.L * wl.Hq * wl.d * 2 / 1e9
+    return {"workload": wl.name, "L": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
+            "layers": f"1 full + {wl.n_sparse} sparse", "topk": wl.topk, "recent": wl.recent,
+            "block": wl.block, "batch_per_gpu": 1, "parallelism": f"independent sequence per GPU x{world}",
+            "l2": "inputs larger than L2 (Q alone is %.1f GB); no flush" % q_gb}
+
+
 def data_recipe(wl) -> str:
     """One line naming the synthetic input recipe of a workload."""
     k = "K from a 64-component Gaussian mixture, std 0.3" if wl.k_dist == "gmm64" else "Q/K/V ~ N(0,1)"
@@ -493,10 +502,7 @@ def run_cuda(args, wl, rank, world, dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 Q, e4m3 K/V (f16 MMA)" if fp8_cache else "bf16",
         "data": data_recipe(wl),
-        "config": {"workload": wl.name, "L": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
-                   "layers": f"1 full + {wl.n_sparse} sparse", "topk": wl.topk, "recent": wl.recent,
-                   "block": wl.block, "batch_per_gpu": 1, "parallelism": f"independent sequence per GPU x{world}",
-                   "l2": "inputs larger than L2 (Q alone is %.1f GB); no flush" % (q0.numel() * 2 / 1e9)},
+        "config": arm_config(wl, world),
         "roofline": {"kernel": "fa_fwd (kernel 1, dense causal attention + LSE)", "bound": "tensor",
                      "achieved": fa_tflops, "peak": peak, "unit": "TFLOP/s", "frac": fa_tflops / peak,
                      "traffic": recorded_traffic(wl.name) if not fp8_cache else None, "traffic_unit": "bytes per launch (dram read + write, ncu)",
@@ -555,9 +561,8 @@ def run_reference(args, wl, rank, world):
     v = float(np.median(vals))
     return {"metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * wl.L / v, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": wl.name, "L": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
-                       "layers": f"1 full + {wl.n_sparse} sparse"},
+            "vs_baseline": None, "dtype": "f64", "data": data_recipe(wl), "impl": "reference",
+            "config": arm_config(wl, world),
             "cpu_baseline": {"value": v, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
                              "sample": "per step: seeded (query block, KV head) units, extrapolated by FLOP ratio"},
             "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -43,3 +43,10 @@ def test_data_recipe_names_each_workloads_inputs():
     assert "8 multi-hop needle chains of 4 keys" in r["c4"]
     assert "e4m3" in r["c5"] and "1024 planted needle keys per KV head" in r["c5"]
     assert all(v.startswith("synthetic (seeded ") for v in r.values())
+
+
+def test_both_arms_share_one_config():
+    wl = inputs.WORKLOADS["c3"]
+    c = bench.arm_config(wl, 1)
+    assert c["workload"] == wl.name and c["L"] == 131072 and c["topk"] == 1024 and c["recent"] == 128
+    assert "2.1 GB" in c["l2"] and c["parallelism"].endswith("x1")
