@@ -472,7 +472,7 @@ def run_cuda(args, wl, rank, world, dist):
         del o_sp, out
         torch.cuda.empty_cache()
         pipe = PrefillPipeline(shape, wl.n_sparse, dev)
-        n_e2e = max(6, args.steps)  # the pipeline's fill and drain are paid once per run
+        n_e2e = max(12, args.steps)  # the pipeline's fill and drain are paid once per run
         for _ in range(2):  # warm-up: both buffer sets once
             pipe.submit(h_q, h_k, h_v, h_o, h_idx, h_cnt)
         pipe.synchronize()
