@@ -609,8 +609,10 @@ def run_stage(args, wl):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
-    ap.add_argument("--warmup", type=int, default=3)
+    # defaults: 10 warm-up and 20 timed steps, median and P99 reported (the MiMo-V3
+    # prefill blog's measurement procedure, section 3.3)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", default="c3", help="c1..c5 (default c3, the 128k workload)")
     ap.add_argument("--no-e2e", action="store_true")
