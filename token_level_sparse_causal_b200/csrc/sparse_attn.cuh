@@ -647,23 +647,33 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         }
         tc_fence_after();
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        // O in two halves of 64 columns, one TMEM wait each; once the second
+        // half is in registers the next item's P V may overwrite O, so o_free
+        // is signalled before the last stores
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t orr[32];
-          tmem_ld32(o_tm + c * 32, orr);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t orr[2][32];
+          tmem_ld32(o_tm + (2 * half) * 32, orr[0]);
+          tmem_ld32(o_tm + (2 * half + 1) * 32, orr[1]);
           tmem_ld_wait();
-          reg_fence(orr);
-          uint32_t pk[16];
+          reg_fence(orr[0]);
+          reg_fence(orr[1]);
+          if (half == 1) {
+            tc_fence_before();
+            mbar_arrive(&bars->o_free[x]);
+          }
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(orr[cc][2 * e]) * inv, __uint_as_float(orr[cc][2 * e + 1]) * inv);
+            uint4* dst = reinterpret_cast<uint4*>(orow + (2 * half + cc) * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
         }
-        tc_fence_before();
-        mbar_arrive(&bars->o_free[x]);
         if (WIN && p.lse != nullptr)  // natural-log LSE of the row
           p.lse[static_cast<int64_t>(hh) * p.L + i_row] = (m_used + log2f(l)) * 0.69314718055994530942f;
       } else if (w.nt == 0 && row_live) {
