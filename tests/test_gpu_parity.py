@@ -493,6 +493,11 @@ def test_fp8_layer_copy_equals_in_kernel_conversion(L, Hq, Hkv):
     hs2.hs2_attn_fwd_ws(shape, q0, k, v, ks, vs, o2, lse2, ws1)
     hs2.hs2_sync()
     assert torch.equal(o2, o1) and torch.equal(lse2, lse1)
+    # a workspace too small for the copy: the kernel converts the tiles itself
+    o3, lse3 = torch.empty_like(q0), torch.empty((Hq, L), device=DEV, dtype=torch.float32)
+    hs2.hs2_attn_fwd_ws(shape, q0, k, v, ks, vs, o3, lse3, torch.empty(4, device=DEV, dtype=torch.float32))
+    hs2.hs2_sync()
+    assert torch.equal(o3, o1) and torch.equal(lse3, lse1)
 
 
 # -------------------------------------------------- device-side failures --
