@@ -500,6 +500,31 @@ def test_fp8_layer_copy_equals_in_kernel_conversion(L, Hq, Hkv):
     assert torch.equal(o3, o1) and torch.equal(lse3, lse1)
 
 
+@pytest.mark.parametrize("L,Hq,Hkv", [(4096, 8, 2), (2560, 16, 2)])
+def test_strip_sizes_do_not_change_the_result(L, Hq, Hkv):
+    """The full-layer call groups query blocks into strips that fit the
+    workspace: the minimum (one block per strip), a few blocks per strip, and
+    the recommended size must all give the same bits."""
+    wl = _wl(L, Hq, Hkv, n_sparse=0, seed=41)
+    xd = H.to_dev(inputs.make_inputs(wl), DEV)
+    shape = H.shape_of(wl, xd)
+    q0, k, v = xd["q_layers"][0], xd["k"], xd["v"]
+    nb = L // 64
+    row = (L - 128 + 63) // 64 * 64 * 4
+    outs = []
+    for nbytes in (Hkv * row, 5 * Hkv * row + 64, hs2.workspace_bytes(shape)):
+        o, lse = torch.empty_like(q0), torch.empty((Hq, L), device=DEV, dtype=torch.float32)
+        idx = torch.empty((Hkv, nb, wl.topk + wl.recent), device=DEV, dtype=torch.int32)
+        cnt = torch.empty((Hkv, nb), device=DEV, dtype=torch.int32)
+        ws = torch.empty(nbytes // 4, device=DEV, dtype=torch.float32)
+        hs2.hs2_full_attn_select(shape, q0, k, v, None, None, o, lse, idx, cnt, ws)
+        hs2.hs2_sync()
+        outs.append((o, lse, idx, cnt))
+    for other in outs[1:]:
+        for a, b in zip(outs[0], other):
+            assert torch.equal(a, b)
+
+
 # -------------------------------------------------- device-side failures --
 
 def test_bounded_wait_reports_timeout_and_context_survives():
