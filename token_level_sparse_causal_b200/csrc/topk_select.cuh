@@ -308,15 +308,16 @@ struct SelSmem {
 
 // Kernel (3).  For rows with n > k candidates, the fast path reads the row
 // once: a sample of up to SEL_SAMPLES values (groups of 8 consecutive values
-// spread evenly over the row) gives a threshold tau (the
-// sample's q-th largest, q chosen so that about 2k values are expected at
-// or above it; tau = 0 when the whole row fits in shared memory), every
-// value >= tau is gathered into shared memory, and there the k-th largest T
-// and the tie count are found exactly, and only the k winners are sorted by
-// position (bitonic; ties at T sorted first when not all of them fit).  The k-th
-// largest of the row is >= tau whenever at least k values were gathered, so
-// the set is exactly the one of the three-pass radix path below; that path
-// runs instead when fewer than k or more than SEL_CAP values were gathered.
+// spread evenly over the row) gives a threshold tau (a lower bound, within
+// 2^10 key steps, of the sample's q-th largest, q chosen so that about 2k
+// values are expected at or above it; tau = 0 when the whole row fits in
+// shared memory), every value >= tau is gathered into shared memory, and
+// there the k-th largest T and the tie count are found exactly; the winners
+// are emitted through a position bitmap, or sorted bitonically for very long
+// rows and for ties at T that do not all fit.  The k-th largest of the row is
+// >= tau whenever at least k values were gathered, so the set is exactly the
+// one of the three-pass radix path below; that path runs instead when fewer
+// than k or more than SEL_CAP values were gathered.
 __global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const SelParams p) {
   extern __shared__ __align__(16) uint8_t sel_raw[];
   SelSmem& S = *reinterpret_cast<SelSmem*>(sel_raw);
