@@ -322,6 +322,23 @@ def select_alone(hs2, torch, shape, q0, k, ks, out, dev, timed, nblk=256):
             "frac_of_hbm": moved / (ms / 1e3) / 1e9 / measured_peaks()["hbm_gbs"]}
 
 
+def importance_alone(hs2, torch, shape, q0, k, ks, out, dev, timed, nblk=256):
+    """Kernel (2) by itself on the last `nblk` query blocks (the longest rows,
+    one launch): device time and the importance FLOP it computes."""
+    nb = shape.L // shape.block
+    b0 = max(0, nb - nblk)
+    G = shape.Hq // shape.Hkv
+    n_c = lambda b: max(0, min(shape.L, shape.block * (b + 1)) - shape.recent)
+    stride = max(4, (n_c(nb - 1) + 3) // 4 * 4)
+    imp = torch.empty((shape.Hkv, nb - b0, stride), dtype=torch.float32, device=dev)
+    ms = timed(lambda: hs2.hs2_importance(shape, q0, k, ks, out["lse"], b0, nb, imp, stride), 3)
+    flop = 2.0 * shape.d * shape.block * G * shape.Hkv * sum(n_c(b) for b in range(b0, nb))
+    hs2.hs2_sync()
+    del imp
+    return {"blocks": [b0, nb], "ms": ms, "flop": flop, "tflops": flop / (ms / 1e3) / 1e12,
+            "frac_of_sustained_bf16": flop / (ms / 1e3) / 1e12 / measured_peaks()["bf16_tflops_sustained"]}
+
+
 DECODE_BATCHES = (1, 128)   # decode queries per call: one token, and a batch at random positions
 
 
@@ -571,8 +588,9 @@ def run_reference(args, wl, rank, world):
 def run_stage(args, wl):
     """One stage alone on a reduced-footprint copy of the workload (same L and
     input recipe, the heads given by --heads, no sparse layers) -- the case
-    an ncu capture of that stage's kernel runs on.  select: kernel (1) for
-    the LSE, then kernel (3) alone on the strip of the longest rows."""
+    an ncu capture of that stage's kernel runs on.  Kernel (1) for the LSE,
+    then kernel (3) (select) or kernel (2) (importance) alone on the strip of
+    the longest rows."""
     import torch
     from token_level_sparse_causal_b200 import build, hs2, inputs
 
@@ -601,9 +619,12 @@ def run_stage(args, wl):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / n
 
-    res = select_alone(hs2, torch, shape, q0, k, ks, out, dev, timed)
+    if args.stage == "importance":
+        res = importance_alone(hs2, torch, shape, q0, k, ks, out, dev, timed)
+    else:
+        res = select_alone(hs2, torch, shape, q0, k, ks, out, dev, timed)
     hs2.hs2_sync(stream)
-    return {"stage": "select_alone", "workload": my.name, "L": my.L, "Hq": hq, "Hkv": hkv, **res}
+    return {"stage": f"{args.stage}_alone", "workload": my.name, "L": my.L, "Hq": hq, "Hkv": hkv, **res}
 
 
 def main(argv=None):
@@ -618,7 +639,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample size for cpu_baseline")
-    ap.add_argument("--stage", choices=["select"], help="time one stage alone (1 GPU) and print its line")
+    ap.add_argument("--stage", choices=["select", "importance"], help="time one stage alone (1 GPU) and print its line")
     ap.add_argument("--heads", help="with --stage: query/KV heads of the reduced copy, e.g. 16/8")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "cuda":
