@@ -168,7 +168,12 @@ int hs2_sync(void* stream);
 
 /* ---- stage-level entry points (same kernels as above, one stage each) ---- */
 
-/* Full causal attention forward with LSE only (kernel 1 of the path). */
+/*
+ * Full causal attention forward with LSE only (kernel 1 of the path).  With an
+ * e4m3 cache the kernel converts every K/V tile it loads (no scratch memory);
+ * hs2_attn_fwd_ws below converts the cache once instead, as the full layer
+ * does.  Both give the same bits.
+ */
 int hs2_attn_fwd(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
                  const float* v_scale, void* o, float* lse, void* stream);
 
