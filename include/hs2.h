@@ -195,7 +195,8 @@ int hs2_attn_fwd_ws(const hs2_shape* shape, const void* q, const void* k, const 
  * layer's lse.  Row (g, b) holds I_j for j in C_b = [0, e_b - recent) at
  * imp[((g * (b1 - b0)) + (b - b0)) * row_stride + j]; entries past |C_b| are
  * not written.  row_stride (floats) must be a multiple of 4 and at least
- * |C_{b1-1}|.
+ * |C_{b1-1}|.  One call covers at most 65535 rows (Hkv * (b1 - b0)), else
+ * HS2_ERR_UNSUPPORTED; hs2_full_attn_select splits its strips accordingly.
  */
 int hs2_importance(const hs2_shape* shape, const void* q, const void* k, const float* k_scale,
                    const float* lse, int32_t b0, int32_t b1, float* imp, int64_t row_stride, void* stream);

@@ -141,6 +141,17 @@ def test_block_ranges_and_strides_rejected(lib):
     assert lib.hs2_topk_select(s, P, 4096, -1, 4, P, P, st) == hs2.HS2_ERR_INVALID_ARG
 
 
+def test_importance_launch_rows_are_capped(lib):
+    """One importance launch covers at most 65535 (KV head, block) rows (its
+    grid's y extent): a wider range is refused before anything is launched."""
+    L, Hkv = 524288, 8
+    s = ctypes.byref(_shape(L=L, Hq=16, Hkv=Hkv, q_tok_stride=16 * 128, kv_tok_stride=Hkv * 128))
+    st = ctypes.c_void_p(0)
+    nb = L // 64
+    assert Hkv * nb > 65535
+    assert lib.hs2_importance(s, P, P, None, P, 0, nb, P, L, st) == hs2.HS2_ERR_UNSUPPORTED
+
+
 def test_workspace_too_small_rejected(lib):
     s = _shape()
     n = ctypes.c_size_t(2 * (2048 - 128) * 4 - 16)

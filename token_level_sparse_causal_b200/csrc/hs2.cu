@@ -497,6 +497,8 @@ size_t min_workspace(const hs2_shape* s) {
 }
 
 constexpr size_t kStripCap = size_t(64) << 20;  // keep one strip L2-resident
+// Rows (KV heads x blocks) of one importance launch: its grid's y extent.
+constexpr int64_t kMaxStripRows = 65535;
 
 // Rows a select launch should have at least: two per SM of a B200 (148 SMs),
 // so that the per-row latency of long rows is overlapped across the GPU.
@@ -635,6 +637,7 @@ int hs2_importance(const hs2_shape* shape, const void* q, const void* k, const f
   if (b0 < 0 || b1 > nb || b0 >= b1) return HS2_ERR_INVALID_ARG;
   if (row_stride % 4 || row_stride < n_cand(shape, b1 - 1)) return HS2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(imp)) return HS2_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(shape->Hkv) * (b1 - b0) > kMaxStripRows) return HS2_ERR_UNSUPPORTED;
   return launch_importance(shape, q, k, k_scale, lse, b0, b1, imp, row_stride, -1,
                            static_cast<cudaStream_t>(stream));
 }
@@ -737,7 +740,9 @@ int full_attn_select_impl(const hs2_shape* shape, const void* q, const void* k, 
       while (b1 < nb && n_cand(shape, b1) <= shape->topk) ++b1;
       if ((rc = launch_select(shape, imp, 64, b, b1, idx, cnt, st))) return rc;
     } else {
-      while (b1 < nb && static_cast<size_t>(shape->Hkv) * (b1 + 1 - b) * strip_stride(shape, b1) * 4u <= ws) ++b1;
+      while (b1 < nb && static_cast<int64_t>(shape->Hkv) * (b1 + 1 - b) <= kMaxStripRows &&
+             static_cast<size_t>(shape->Hkv) * (b1 + 1 - b) * strip_stride(shape, b1) * 4u <= ws)
+        ++b1;
       const int64_t stride = strip_stride(shape, b1 - 1);
       if ((rc = launch_importance(shape, q, k, k_scale, lse, b, b1, imp, stride, shape->topk, st, dq))) return rc;
       if ((rc = launch_select(shape, imp, stride, b, b1, idx, cnt, st, blocks))) return rc;
