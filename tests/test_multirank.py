@@ -53,7 +53,7 @@ def test_single_rank_needs_no_group():
     assert bench.reduce_max(3.5, None) == 3.5
 
 
-def test_work_accounting_matches_the_scope_table():
+def test_work_accounting_matches_the_exact_causal_counts():
     """Exact causal counts for the 128k workload (FLOP and bytes per the
     formulas FA = Hq*4d*L(L+1)/2, importance = Hq*64*2d*sum|C_b|)."""
     w = bench.algorithmic_work(inputs.WORKLOADS["c3"])
