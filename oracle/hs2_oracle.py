@@ -20,8 +20,7 @@ Sources (pages, cited by title and paragraph or section):
   [SHARP] "企业官网建设流程全解析" (a walk-through of SHARP sparse attention),
           section 1.1: Attention(Q,K,V) = softmax(Q K^T / sqrt(d_k)) V.
 
-Readings where the pages are silent (each one is also listed in the design
-notes of this repository):
+Readings where the pages are silent:
   R1  scores are s = q.k / sqrt(d), natural-log LSE;
   R2  grouped-query attention maps query head h to KV head floor(h / G);
   R3  one selection per (query block of 64 tokens, KV head), shared by the
