@@ -9,11 +9,14 @@ layers (its Q/K/V/O tensors are far larger than the 126 MB L2, so no flush is
 needed between steps).
 
   python bench.py [--gpus N --steps K --warmup W] [--impl cuda|reference]
+                  [--workload c1..c5] [--stage select|importance --heads HQ/HKV]
 
-Under torchrun every rank runs its own independent sequence (weak scaling,
-no collective on the data path); the step time is the max over ranks.
+Defaults: 10 warm-up and 20 timed steps (median and P99 reported).  Under
+torchrun every rank runs its own independent sequence (weak scaling, no
+collective on the data path); the step time is the max over ranks.
 `--impl reference` times the fp64 CPU oracle on a bounded sample instead.
-Prints one JSON line on rank 0.
+`--stage` times one kernel alone on a reduced-head copy of the workload (the
+case its ncu capture runs on).  Prints one JSON line on rank 0.
 """
 from __future__ import annotations
 
