@@ -574,3 +574,26 @@ def test_decode_hand_case_and_empty_visibility():
     assert np.abs(O[0, 0] - want).max() < 1e-15
     O2 = orc.sparse_decode(q, np.array([2]), K, V, idx, cnt, 64)
     assert np.all(O2 == 0.0)
+
+
+def test_swa_and_decode_planted_mistakes_are_caught():
+    """Plausible bugs in the window and decode oracles, each rejected by the
+    pin above that targets it: a window one key wider (i - W <= j), a decode
+    query that reads the next block's list, and one with no causal mask."""
+    L, Hq, Hkv, d = 150, 4, 2, 16
+    Q, K, V = _rand((L, Hq, d), 71), _rand((L, Hkv, d), 72), _rand((L, Hkv, d), 73)
+    i, j = np.arange(L)[:, None], np.arange(L)[None, :]
+    W = 7
+    band = np.broadcast_to((j <= i) & (j > i - W), (Hq, L, L)).copy()
+    O_wide, _ = orc.swa_attn(Q, K, V, W + 1)           # mutant: one key wider
+    assert np.abs(O_wide - _sdpa(Q, K, V, mask=band)).max() > 1e-3
+
+    L, Hq, Hkv, d, B = 192, 4, 2, 16, 64
+    Q, K, V = _rand((L, Hq, d), 81), _rand((L, Hkv, d), 82), _rand((L, Hkv, d), 83)
+    idx, cnt = _full_lists(L, Hkv, B)
+    pos = np.array([1, 63, 64, 100])
+    ref = _sdpa(Q, K, V, causal=True)[pos]
+    O_next = orc.sparse_decode(Q[pos], pos + B, K, V, idx, cnt, B)   # mutant: next block's list
+    assert np.abs(O_next - ref).max() > 1e-3
+    O_nomask = orc.sparse_decode(Q[pos], np.full_like(pos, L - 1), K, V, idx, cnt, B)  # mutant: no j <= t
+    assert np.abs(O_nomask - ref).max() > 1e-3
