@@ -249,34 +249,30 @@ def select(I_row, k: int, w: int, e_b: int):
     return idx, int(chosen.size)
 
 
-def pool_blocks_fp32(I_row, B: int = 64):
-    """Per-64-key-block sums of an fp32 importance row, in the fixed float32
-    order this library defines for block-level selection: each of 16 lanes
-    adds its 4 consecutive values left to right, then the 16 partial sums are
-    combined by a butterfly (lane l adds lane l ^ 8, then ^ 4, ^ 2, ^ 1; the
-    sum is commutative at every step, so all lanes agree).  Returns float32."""
+def pool_blocks(I_row, B: int = 64):
+    """Importance of each whole 64-key block: the exact sum of its 64 values,
+    taken in float64 (the block-level selection of [HS2]'s block-selection
+    paragraph ranks blocks by how much of the row's importance they hold; the
+    page fixes no summation order, so the oracle sums in float64, where the
+    rounding of 64 float32 terms is far below any float32 difference)."""
     assert B == 64
-    x = np.asarray(I_row, dtype=np.float32).reshape(-1, 16, 4)
-    a = ((x[:, :, 0] + x[:, :, 1]) + x[:, :, 2]) + x[:, :, 3]
-    lanes = np.arange(16)
-    for o in (8, 4, 2, 1):
-        a = (a + a[:, lanes ^ o]).astype(np.float32)
-    return a[:, 0]
+    x = np.asarray(I_row, dtype=np.float64)
+    return x.reshape(-1, B).sum(axis=1)
 
 
 def select_blocks(I_row, k: int, w: int, e_b: int, B: int = 64):
     """Block-level selection of HySparse v1 ([HS2] block-selection paragraph:
     whole 64-token blocks are chosen) on the same importance, as the variant
     the token-level design is compared with: the candidates C_b are pooled
-    into 64-key blocks (pool_blocks_fp32), the top min(#blocks, k / 64) blocks
-    by pooled importance are kept (ties to the lower block), their positions
+    into 64-key blocks (pool_blocks), the top min(#blocks, k / 64) blocks by
+    pooled importance are kept (ties to the lower block), their positions
     listed in ascending order, and the recent window appended; -1 padded to
     k + w.  Requires k % 64 == 0 and |C_b| % 64 == 0."""
     n_c = n_candidates(e_b, w)
     assert k % B == 0 and n_c % B == 0
-    I_row = np.asarray(I_row, dtype=np.float32)
+    I_row = np.asarray(I_row, dtype=np.float64)
     assert I_row.shape == (n_c,)
-    J = pool_blocks_fp32(I_row, B).astype(np.float64) if n_c else np.zeros(0)
+    J = pool_blocks(I_row, B) if n_c else np.zeros(0)
     m = np.arange(J.size)
     order = np.lexsort((m, -J))
     keep = np.sort(order[: min(J.size, k // B)])

@@ -1,6 +1,15 @@
 """Block-level selection (HySparse v1) on the GPU against the oracle's
-select_blocks, bit-exact on the same exported fp32 importance; and the needle
-recall of both granularities on the 32k workload (reported, not a pin)."""
+select_blocks, on the same exported fp32 importance.
+
+The oracle pools each 64-key block in float64; the GPU sums the same 64 fp32
+values in fp32.  For nonnegative terms, any fp32 summation order of n terms is
+within gamma_{n-1} * sum of the exact sum (Higham, "Accuracy and Stability of
+Numerical Algorithms", Lemma 8.4), gamma_m = m u / (1 - m u), u = 2^-24.  So the
+GPU can rank block x below block y only if J_x - J_y <= gamma_63 (J_x + J_y).
+The lists must equal the oracle's bit for bit unless such a near-tie straddles
+the top-(k/64) boundary; then every GPU choice must be one the bound allows.
+Rows whose block sums are exact in fp32 (crafted tie rows) are compared bit for
+bit, which pins the tie rule (lower block first)."""
 import numpy as np
 import pytest
 import torch
@@ -11,6 +20,8 @@ from token_level_sparse_causal_b200 import hs2, inputs
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
+U = 2.0 ** -24
+GAMMA63 = 63 * U / (1 - 63 * U)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -21,31 +32,51 @@ def _built():
     hs2.hs2_debug_set(H.WAIT_LIMIT_NS, 0)
 
 
-def _path_blocks(wl, xd):
-    q0, k, v = xd["q_layers"][0], xd["k"], xd["v"]
-    shape = H.shape_of(wl, xd)
-    out = hs2.alloc_outputs(shape, q0)
-    hs2.hs2_full_attn_select_blocks(shape, q0, k, v, xd.get("k_scale"), xd.get("v_scale"), out["o"], out["lse"],
-                                    out["idx"], out["cnt"], out["workspace"])
-    hs2.hs2_sync()
-    return shape, out
+def check_block_list(row32, idx, cnt, k, w, e_b, exact=False):
+    """Returns 'exact' when the GPU list equals the oracle's, 'near-tie' when
+    it differs only where the fp32 rounding bound allows; asserts otherwise."""
+    want, wc = orc.select_blocks(row32, k, w, e_b)
+    assert cnt == wc, (cnt, wc)
+    assert np.all(idx[cnt:] == -1)
+    if np.array_equal(idx, want):
+        return "exact"
+    assert not exact, "rows with exact fp32 block sums must match bit for bit"
+    nrec = min(w, e_b)
+    assert np.array_equal(idx[cnt - nrec:cnt], want[wc - nrec:wc]), "recent window"
+    glob = idx[:cnt - nrec].reshape(-1, 64)
+    blocks = glob[:, 0] // 64
+    assert np.all(glob == blocks[:, None] * 64 + np.arange(64)[None, :]), "whole blocks"
+    assert np.all(np.diff(blocks) > 0), "ascending, distinct"
+    J = orc.pool_blocks(row32)
+    chosen = np.zeros(J.size, bool)
+    chosen[blocks] = True
+    for x in np.flatnonzero(chosen):
+        beat = (~chosen) & (J - J[x] > GAMMA63 * (J + J[x]))
+        assert not beat.any(), f"block {int(np.flatnonzero(beat)[0])} beats chosen block {x} beyond rounding"
+    return "near-tie"
 
 
 @pytest.mark.parametrize("L,Hq,Hkv", [(4096, 8, 2), (2304, 8, 1)])
-def test_block_path_bit_exact_on_exported_importance(L, Hq, Hkv):
+def test_block_path_matches_fp64_oracle_on_exported_importance(L, Hq, Hkv):
     wl = inputs.Workload(f"b{L}", L, Hq, Hkv, 1, seed=41)
     x = inputs.make_inputs(wl)
     xd = H.to_dev(x, DEV)
-    shape, out = _path_blocks(wl, xd)
+    q0, k, v = xd["q_layers"][0], xd["k"], xd["v"]
+    shape = H.shape_of(wl, xd)
+    out = hs2.alloc_outputs(shape, q0)
+    hs2.hs2_full_attn_select_blocks(shape, q0, k, v, None, None, out["o"], out["lse"], out["idx"], out["cnt"],
+                                    out["workspace"])
+    hs2.hs2_sync()
     nb = L // 64
     imp = H.gpu_importance(shape, xd, out["lse"], 0, nb).cpu().numpy()
     idx, cnt = out["idx"].cpu().numpy(), out["cnt"].cpu().numpy()
+    kinds = []
     for b in range(nb):
         _, e_b = orc.block_rows(b, L, 64)
         n_c = orc.n_candidates(e_b, 128)
         for g in range(Hkv):
-            want, wc = orc.select_blocks(imp[g, b, :n_c], 1024, 128, e_b)
-            assert cnt[g, b] == wc and np.array_equal(idx[g, b], want), (g, b)
+            kinds.append(check_block_list(imp[g, b, :n_c], idx[g, b], int(cnt[g, b]), 1024, 128, e_b))
+    assert kinds.count("exact") >= 0.95 * len(kinds), kinds.count("near-tie")
 
 
 def test_block_select_crafted_rows():
@@ -59,7 +90,7 @@ def test_block_select_crafted_rows():
     rows = np.zeros((Hkv, b1 - b0, stride), np.float32)
     for bi, b in enumerate(range(b0, b1)):
         n = orc.n_candidates(64 * (b + 1), 128)
-        rows[0, bi, :n] = (rng.integers(0, 3, n) / 4).astype(np.float32)       # heavy ties between blocks
+        rows[0, bi, :n] = (rng.integers(0, 3, n) / 4).astype(np.float32)       # heavy exact ties between blocks
         rows[1, bi, :n] = 1.0                                                  # all blocks equal
         rows[2, bi, :n] = rng.random(n).astype(np.float32)
         rows[3, bi, :n] = np.exp(-rng.random(n) * 60).astype(np.float32)
@@ -72,24 +103,7 @@ def test_block_select_crafted_rows():
         e_b = 64 * (b + 1)
         n = orc.n_candidates(e_b, 128)
         for g in range(Hkv):
-            want, wc = orc.select_blocks(rows[g, bi, :n], 1024, 128, e_b)
-            assert int(cnt[g, b]) == wc and np.array_equal(idx[g, b].cpu().numpy(), want), (g, b)
-
-
-def test_needle_recall_token_vs_block_on_32k():
-    wl = inputs.WORKLOADS["c2"]
-    xd = inputs.make_inputs(wl, device=DEV)
-    r_tok = H.run_path(wl.scaled(n_sparse=0), {**xd, "q_layers": xd["q_layers"][:1]})
-    _, r_blk = _path_blocks(wl, xd)
-
-    def recall(idx, cnt):
-        hit = 0
-        for n in xd["needles"]:
-            b = n["t"] // 64
-            lst = idx[n["g"], b, :cnt[n["g"], b]]
-            hit += int(n["p"] in set(lst.tolist()))
-        return hit / len(xd["needles"])
-    rt = recall(r_tok["idx"].cpu().numpy(), r_tok["cnt"].cpu().numpy())
-    rb = recall(r_blk["idx"].cpu().numpy(), r_blk["cnt"].cpu().numpy())
-    print(f"needle recall on the 32k workload: token-level {rt:.4f}, block-level {rb:.4f}")
-    assert 0.0 <= rb <= 1.0 and 0.0 <= rt <= 1.0
+            # rows 0 and 1 hold multiples of 1/4 below 2^7: every partial sum is
+            # exact in fp32, so the GPU's sums equal the oracle's
+            check_block_list(rows[g, bi, :n], idx[g, b].cpu().numpy(), int(cnt[g, b]), 1024, 128, e_b,
+                             exact=g < 2)

@@ -438,20 +438,30 @@ def test_quantize_kv_row_definition():
 
 # ------------------------------------------------ block-level selection (v1) --
 
-def test_pool_blocks_tree_is_a_sum():
+def _fsum_blocks(I, B=64):
+    """Correctly rounded per-block sums by math.fsum over plain Python floats:
+    a routine that shares nothing with the oracle's vectorised float64 sum."""
+    vals = [float(x) for x in np.asarray(I, np.float32)]
+    return [math.fsum(vals[m * B:(m + 1) * B]) for m in range(len(vals) // B)]
+
+
+def test_pool_blocks_is_the_block_sum():
     rng = np.random.default_rng(9)
-    I = rng.random(64 * 37).astype(np.float32)
-    J = orc.pool_blocks_fp32(I)
-    ref = I.astype(np.float64).reshape(-1, 64).sum(axis=1)
-    assert J.dtype == np.float32 and np.all(np.abs(J - ref) <= 64 * 2.0 ** -24 * ref)
+    for I in (rng.random(64 * 37).astype(np.float32),
+              np.exp(-rng.random(64 * 23) * 80).astype(np.float32),     # 35 binades in one block
+              (rng.integers(0, 5, 64 * 11) / 8).astype(np.float32)):
+        J = orc.pool_blocks(I)
+        ref = np.array(_fsum_blocks(I))
+        assert J.dtype == np.float64 and np.all(np.abs(J - ref) <= 1e-14 * ref)
     Iz = np.zeros(64 * 3, np.float32)
-    Iz[64 + 7] = 3.0                                   # exact in any order
-    assert list(orc.pool_blocks_fp32(Iz)) == [0.0, 3.0, 0.0]
+    Iz[64 + 7] = 3.0
+    assert list(orc.pool_blocks(Iz)) == [0.0, 3.0, 0.0]
 
 
 def check_select_blocks_brute(sel_fn, seed=0):
     """Brute force at block granularity: block m is kept iff fewer than k/64
-    blocks beat it (higher pooled value, or equal and lower index)."""
+    blocks beat it (higher pooled value, or equal and lower index), with the
+    pooled values from math.fsum."""
     rng = np.random.default_rng(seed)
     k, w, B = 256, 128, 64
     bad = 0
@@ -459,11 +469,15 @@ def check_select_blocks_brute(sel_fn, seed=0):
         for b in range(L // B):
             e_b = B * (b + 1)
             n_c = orc.n_candidates(e_b, w)
-            I = (rng.integers(0, 3, n_c) / 2.0).astype(np.float32)
+            if seed % 2:
+                I = (rng.integers(0, 3, n_c) / 2.0).astype(np.float32)       # many exact block ties
+            else:
+                I = rng.random(n_c).astype(np.float32)
             idx, cnt = sel_fn(I, k, w, e_b)
-            J = orc.pool_blocks_fp32(I).astype(np.float64) if n_c else np.zeros(0)
-            rank = orc.brute_rank(J)
-            want = [p for m in range(J.size) if rank[m] < k // B for p in range(m * B, (m + 1) * B)]
+            J = _fsum_blocks(I)
+            nbk = len(J)
+            rank = [sum(1 for m2 in range(nbk) if J[m2] > J[m] or (J[m2] == J[m] and m2 < m)) for m in range(nbk)]
+            want = [p for m in range(nbk) if rank[m] < k // B for p in range(m * B, (m + 1) * B)]
             want += list(range(max(0, e_b - w), e_b))
             bad += int(list(idx[:cnt]) != want) + int(np.any(idx[cnt:] != -1))
     return bad
@@ -481,7 +495,7 @@ def test_select_blocks_brute_force_and_sizes():
 def test_select_blocks_planted_mistake_is_caught():
     def ties_high(I, k, w, e_b, B=64):
         n_c = orc.n_candidates(e_b, w)
-        J = orc.pool_blocks_fp32(np.asarray(I, np.float32)).astype(np.float64) if n_c else np.zeros(0)
+        J = orc.pool_blocks(I) if n_c else np.zeros(0)
         m = np.arange(J.size)
         keep = np.sort(np.lexsort((-m, -J))[:min(J.size, k // B)])
         top = (keep[:, None] * B + np.arange(B)[None, :]).reshape(-1)
@@ -489,7 +503,18 @@ def test_select_blocks_planted_mistake_is_caught():
         idx = np.full(k + w, -1, np.int64)
         idx[:ch.size] = ch
         return idx, ch.size
-    assert check_select_blocks_brute(ties_high) > 0
+    assert check_select_blocks_brute(ties_high, seed=1) > 0
+
+    def first_value_only(I, k, w, e_b, B=64):        # pools by the block's first key instead of its sum
+        n_c = orc.n_candidates(e_b, w)
+        J = np.asarray(I, np.float64)[::B] if n_c else np.zeros(0)
+        keep = np.sort(np.lexsort((np.arange(J.size), -J))[:min(J.size, k // B)])
+        ch = np.concatenate([(keep[:, None] * B + np.arange(B)[None, :]).reshape(-1),
+                             np.arange(max(0, e_b - w), e_b)])
+        idx = np.full(k + w, -1, np.int64)
+        idx[:ch.size] = ch
+        return idx, ch.size
+    assert check_select_blocks_brute(first_value_only, seed=0) > 0
 
 
 # ------------------------------------------------- sliding-window attention --
