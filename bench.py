@@ -9,14 +9,16 @@ layers (its Q/K/V/O tensors are far larger than the 126 MB L2, so no flush is
 needed between steps).
 
   python bench.py [--gpus N --steps K --warmup W] [--impl cuda|reference]
-                  [--workload c1..c5] [--stage select|importance --heads HQ/HKV]
+                  [--workload c1..c5] [--stage fa|importance|select|sparse --heads HQ/HKV]
 
 Defaults: 10 warm-up and 20 timed steps (median and P99 reported).  Under
 torchrun every rank runs its own independent sequence (weak scaling, no
 collective on the data path); the step time is the max over ranks.
 `--impl reference` times the fp64 CPU oracle on a bounded sample instead.
-`--stage` times one kernel alone on a reduced-head copy of the workload (the
-case its ncu capture runs on).  Prints one JSON line on rank 0.
+`--stage` times one kernel alone (fa: kernel (1); importance: kernel (2);
+select: kernel (3); sparse: kernel (4), one layer) on a reduced-head copy of
+the workload (the case its ncu capture runs on).  Prints one JSON line on
+rank 0.
 """
 from __future__ import annotations
 
@@ -342,6 +344,20 @@ def importance_alone(hs2, torch, shape, q0, k, ks, out, dev, timed, nblk=256):
             "frac_of_sustained_bf16": flop / (ms / 1e3) / 1e12 / measured_peaks()["bf16_tflops_sustained"]}
 
 
+def needle_recall(needles, idx, cnt, block: int = 64):
+    """Share of planted needle keys that appear in the index list of their
+    target query's block and KV head (a diagnostic of the selection on the
+    workload's retrieval structure, not a parity check)."""
+    if not needles:
+        return None
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    hit = 0
+    for n in needles:
+        b = n["t"] // block
+        hit += int(n["p"] in set(idx_h[n["g"], b, :cnt_h[n["g"], b]].tolist()))
+    return hit / len(needles)
+
+
 DECODE_BATCHES = (1, 128)   # decode queries per call: one token, and a batch at random positions
 
 
@@ -469,9 +485,11 @@ def run_cuda(args, wl, rank, world, dist):
                                               o_sp[0], stream), n_stage) if o_sp else 0.0
     fs_ms = timed(lambda: hs2.hs2_full_attn_select(shape, q0, k, v, ks, vs, out["o"], out["lse"], out["idx"],
                                                    out["cnt"], out["workspace"], stream), n_stage)
+    recall_tok = needle_recall(x.get("needles"), out["idx"], out["cnt"])
     blk_ms = timed(lambda: hs2.hs2_full_attn_select_blocks(shape, q0, k, v, None, None, out["o"], out["lse"],
                                                            out["idx"], out["cnt"], out["workspace"], stream),
                    n_stage) if wl.topk % 64 == 0 and k.dtype == torch.bfloat16 else None
+    recall_blk = needle_recall(x.get("needles"), out["idx"], out["cnt"]) if blk_ms is not None else None
     swa_ms = timed(lambda: hs2.hs2_swa_attn(shape, q0, k, v, SWA_WINDOW, out["o"], None, stream),
                    n_stage) if k.dtype == torch.bfloat16 else None
     decode = decode_rows(hs2, torch, shape, x, k, v, ks, vs, out, dev, timed) if o_sp else None
@@ -542,6 +560,9 @@ def run_cuda(args, wl, rank, world, dist):
         "next_rows": {"fp8_kv_write_K": fp8,
                       "block_level_full_attn_select_ms": blk_ms,
                       "token_level_full_attn_select_ms": fs_ms,
+                      "needle_recall": None if recall_tok is None else {
+                          "token_level": recall_tok, "block_level": recall_blk,
+                          "note": "share of planted needle keys listed for their target block (diagnostic)"},
                       "swa_attn": None if swa_ms is None else {
                           "window": SWA_WINDOW, "ms": swa_ms,
                           "tflops": work["swa_flop"] / (swa_ms / 1e3) / 1e12,
@@ -580,7 +601,10 @@ def run_reference(args, wl, rank, world):
             vals.append(wl.L / (t * total / sum(_unit_flop(wl, b) for b, _ in units)))
     v = float(np.median(vals))
     return {"metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1e3 * wl.L / v, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": 1e3 * wl.L / v, "extrapolated": True,
+            "ms_per_step_note": "whole-prefill time extrapolated from the timed sample by the exact FLOP ratio; "
+                                "the run itself takes about (warmup + steps) x cpu_seconds / 3",
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": data_recipe(wl), "impl": "reference",
             "config": arm_config(wl, world),
             "cpu_baseline": {"value": v, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
@@ -592,8 +616,9 @@ def run_stage(args, wl):
     """One stage alone on a reduced-footprint copy of the workload (same L and
     input recipe, the heads given by --heads, no sparse layers) -- the case
     an ncu capture of that stage's kernel runs on.  Kernel (1) for the LSE,
-    then kernel (3) (select) or kernel (2) (importance) alone on the strip of
-    the longest rows."""
+    then kernel (1) again (fa), kernel (2) (importance) or kernel (3)
+    (select) alone on the strip of the longest rows, or one sparse layer
+    (sparse) on the full layer's lists."""
     import torch
     from token_level_sparse_causal_b200 import build, hs2, inputs
 
@@ -622,8 +647,33 @@ def run_stage(args, wl):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / n
 
+    work = algorithmic_work(my)
+    peaks = measured_peaks()
     if args.stage == "importance":
         res = importance_alone(hs2, torch, shape, q0, k, ks, out, dev, timed)
+    elif args.stage == "fa":
+        # kernel (1) alone, as the full layer runs it
+        fa_ws = None
+        if fp8_cache:
+            fa_ws = torch.empty(hs2.attn_fwd_workspace_bytes(shape) // 4 + 4, dtype=torch.float32, device=dev)
+        ms = timed(lambda: hs2.hs2_attn_fwd_ws(shape, q0, k, v, ks, vs, out["o"], out["lse"], fa_ws, stream), 3)
+        tf = work["fa_flop"] / (ms / 1e3) / 1e12
+        res = {"ms": ms, "flop": work["fa_flop"], "tflops": tf, "frac_of_sustained_bf16": tf / peaks["bf16_tflops_sustained"],
+               "algorithmic_bytes": 2 * my.L * hq * my.d * 2 + 2 * my.L * hkv * my.d * k.element_size() + my.L * hq * 4}
+    elif args.stage == "sparse":
+        # kernel (4) alone: one sparse layer on the full layer's lists
+        hs2.hs2_full_attn_select(shape, q0, k, v, ks, vs, out["o"], out["lse"], out["idx"], out["cnt"],
+                                 out["workspace"], stream)
+        q1 = torch.randn(q0.shape, device=dev, generator=torch.Generator(device=dev).manual_seed(my.seed * 1000 + 1)
+                         ).to(torch.bfloat16)
+        o1 = torch.empty_like(q1)
+        ms = timed(lambda: hs2.hs2_sparse_attn(shape, q1, k, v, ks, vs, out["idx"], out["cnt"], o1, stream), 3)
+        tf = work["sparse_flop"] / (ms / 1e3) / 1e12
+        moved = work["gather_bytes"] + work["sparse_qo_bytes"]
+        res = {"ms": ms, "flop": work["sparse_flop"], "tflops": tf,
+               "frac_of_sustained_bf16": tf / peaks["bf16_tflops_sustained"], "gather_bytes": work["gather_bytes"],
+               "qo_bytes": work["sparse_qo_bytes"], "gbs": moved / (ms / 1e3) / 1e9,
+               "frac_of_hbm": moved / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
     else:
         res = select_alone(hs2, torch, shape, q0, k, ks, out, dev, timed)
     hs2.hs2_sync(stream)
@@ -642,7 +692,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample size for cpu_baseline")
-    ap.add_argument("--stage", choices=["select", "importance"], help="time one stage alone (1 GPU) and print its line")
+    ap.add_argument("--stage", choices=["select", "importance", "fa", "sparse"],
+                    help="time one stage alone (1 GPU) and print its line")
     ap.add_argument("--heads", help="with --stage: query/KV heads of the reduced copy, e.g. 16/8")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "cuda":

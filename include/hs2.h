@@ -38,6 +38,14 @@
  *                                         dimension is contiguous
  *       k/v_scale : fp32 [L][Hkv] contiguous (only for kv_dtype = E4M3:
  *                   stored value = e4m3(code) * scale)
+ *   - With an e4m3 cache (kv_dtype = HS2_KV_E4M3) the tensor-core products run
+ *     on f16 operands: e4m3 codes convert to f16 exactly, and Q is rounded
+ *     from bf16 to f16, which is exact for magnitudes in [2^-14, 65504].
+ *     Smaller magnitudes become f16 subnormals (multiples of 2^-24, so they
+ *     keep fewer bits); a magnitude of 65520 or more has no f16 value, and
+ *     a Q holding one is reported by the next hs2_sync as HS2_ERR_RANGE (the
+ *     outputs of that call are then meaningless).  A bf16 cache has no such
+ *     limit.
  *       lse       : fp32 [Hq][L]  (natural log)
  *       idx       : int32 [Hkv][nb][topk + recent], nb = L / block,
  *                   ascending positions, -1 padded
@@ -69,7 +77,9 @@ enum hs2_status {
   HS2_ERR_WORKSPACE = 3,    /* workspace smaller than the minimum */
   HS2_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
   HS2_ERR_TIMEOUT = 5,      /* a device-side bounded wait ran out */
-  HS2_ERR_INDEX = 6         /* an index list held a position outside [0, e_b) */
+  HS2_ERR_INDEX = 6,        /* an index list held a position outside [0, e_b) */
+  HS2_ERR_RANGE = 7         /* an input value outside the supported range (see
+                               kv_dtype = HS2_KV_E4M3 below) */
 };
 
 enum hs2_kv_dtype { HS2_KV_BF16 = 0, HS2_KV_E4M3 = 1 };
@@ -101,10 +111,27 @@ typedef struct hs2_shape {
  *   the workspace whenever it fits beside the minimum: the cache is then
  *   converted once instead of inside every tile load of the attention and
  *   importance kernels.  Results are identical either way.
+ *
+ * importance_out / strip_b0 / strip_b1: optional export, for checking, of the
+ *   very importance rows the selection consumed.  NULL: no export (strip_b0
+ *   and strip_b1 are ignored).  Otherwise, for the query blocks
+ *   b in [strip_b0, strip_b1) (0 <= strip_b0 < strip_b1 <= L / 64) and every
+ *   KV head g, row (g, b) is copied out of the workspace, after kernel (2)
+ *   wrote it and before the next strip overwrites it, to
+ *     importance_out[((g * (strip_b1 - strip_b0)) + (b - strip_b0)) * S + j],
+ *   j in C_b = [0, e_b - recent), with the row stride
+ *     S = max(64, roundup(e_{strip_b1 - 1} - recent, 64)) floats
+ *   (the Python binding's importance_row_stride computes it).  Entries past
+ *   |C_b| are unspecified; the rows of blocks with |C_b| <= topk (every
+ *   candidate is selected there, so no importance is computed) are left
+ *   untouched.
+ *   importance_out: device memory of Hkv * (strip_b1 - strip_b0) * S floats,
+ *   4-byte aligned; a bad range returns HS2_ERR_INVALID_ARG.
  */
 int hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, const void* v,
                          const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,
-                         int32_t* cnt, void* workspace, size_t* workspace_bytes, void* stream);
+                         int32_t* cnt, void* workspace, size_t* workspace_bytes, float* importance_out,
+                         int32_t strip_b0, int32_t strip_b1, void* stream);
 
 /*
  * hs2_full_attn_select without a caller workspace.  (The paper has no
@@ -220,12 +247,16 @@ int hs2_topk_select(const hs2_shape* shape, const float* imp, int64_t row_stride
  * added left to right, then combined pairwise at distances 8, 4, 2, 1 -- the
  * top topk/64 blocks are kept (ties to the lower block) and listed as
  * ascending positions, followed by the recent window.  Same layouts and list
- * sizes as the token-level lists.  Requires topk % 64 == 0.
+ * sizes as the token-level lists.  Blocks whose sums agree to within the fp32
+ * rounding of a 64-term sum may rank either way.  Requires topk % 64 == 0 and
+ * L <= 2^20 (a row's pooled values are held in 64 KiB of shared memory), else
+ * HS2_ERR_UNSUPPORTED.
  */
 int hs2_block_select(const hs2_shape* shape, const float* imp, int64_t row_stride, int32_t b0, int32_t b1,
                      int32_t* idx, int32_t* cnt, void* stream);
 
-/* hs2_full_attn_select with block-level instead of token-level selection. */
+/* hs2_full_attn_select with block-level instead of token-level selection
+ * (same limits as hs2_block_select; no importance export). */
 int hs2_full_attn_select_blocks(const hs2_shape* shape, const void* q, const void* k, const void* v,
                                 const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,
                                 int32_t* cnt, void* workspace, size_t* workspace_bytes, void* stream);
@@ -287,7 +318,12 @@ const char* hs2_strerror(int code);
  * Limit for every device-side wait, in nanoseconds (default 2e9).  Test hook
  * flags: bit 0 makes the attention kernels' load role issue nothing, so the
  * bounded waits of the other roles must run out and hs2_sync must report
- * HS2_ERR_TIMEOUT.  Flags are 0 in normal use.
+ * HS2_ERR_TIMEOUT.  Bit 1 (checking mode) makes hs2_importance compute each
+ * row over every visible key j < e_b with the causal mask j <= i, not only
+ * over the candidates C_b (row_stride must then be at least e_{b1-1}): such
+ * a row sums to 64 * G (every query's probabilities sum to one), which a test
+ * checks; its first |C_b| entries equal the normal row's.  hs2_full_attn_select
+ * ignores bit 1.  Flags are 0 in normal use.
  */
 int hs2_debug_set(uint64_t wait_limit_ns, uint32_t flags);
 

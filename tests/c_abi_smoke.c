@@ -23,7 +23,7 @@ int main(void) {
   s.kv_head_stride = 128;
 
   size_t ws = 0;
-  int rc = hs2_full_attn_select(&s, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, &ws, NULL);
+  int rc = hs2_full_attn_select(&s, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, &ws, NULL, 0, 0, NULL);
   printf("full_ws_rc %d\nfull_ws_bytes %zu\n", rc, ws);
 
   size_t fa_ws = 123;
@@ -40,7 +40,7 @@ int main(void) {
   printf("decode_ws_rc %d\ndecode_ws_bytes %zu\n", rc, dec_ws);
 
   s.d = 64; /* unsupported head size: refused before any launch */
-  rc = hs2_full_attn_select(&s, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, &ws, NULL);
+  rc = hs2_full_attn_select(&s, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, &ws, NULL, 0, 0, NULL);
   printf("bad_d_rc %d\n", rc);
 
   printf("version %d\n", hs2_version());

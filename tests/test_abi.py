@@ -112,7 +112,7 @@ def test_bad_shapes_rejected(lib, kw, code):
     assert lib.hs2_attn_fwd(s, P, P, P, None, None, P, P, st) == code
     assert lib.hs2_sparse_attn(s, P, P, P, None, None, P, P, P, st) == code
     n = ctypes.c_size_t(1 << 30)
-    assert lib.hs2_full_attn_select(s, P, P, P, None, None, P, P, P, P, P, ctypes.byref(n), st) == code
+    assert lib.hs2_full_attn_select(s, P, P, P, None, None, P, P, P, P, P, ctypes.byref(n), None, 0, 0, st) == code
     assert lib.hs2_importance(s, P, P, None, P, 0, 1, P, 4096, st) == code
     assert lib.hs2_topk_select(s, P, 4096, 0, 1, P, P, st) == code
 
@@ -155,11 +155,27 @@ def test_importance_launch_rows_are_capped(lib):
 def test_workspace_too_small_rejected(lib):
     s = _shape()
     n = ctypes.c_size_t(2 * (2048 - 128) * 4 - 16)
-    rc = lib.hs2_full_attn_select(ctypes.byref(s), P, P, P, None, None, P, P, P, P, P, ctypes.byref(n),
+    rc = lib.hs2_full_attn_select(ctypes.byref(s), P, P, P, None, None, P, P, P, P, P, ctypes.byref(n), None, 0, 0,
                                   ctypes.c_void_p(0))
     assert rc == hs2.HS2_ERR_WORKSPACE
-    assert lib.hs2_full_attn_select(ctypes.byref(s), P, P, P, None, None, P, P, P, P, P, None,
+    assert lib.hs2_full_attn_select(ctypes.byref(s), P, P, P, None, None, P, P, P, P, P, None, None, 0, 0,
                                     ctypes.c_void_p(0)) == hs2.HS2_ERR_INVALID_ARG
+
+
+def test_importance_export_range_checked(lib):
+    """The optional importance export of hs2_full_attn_select takes a block
+    range inside [0, L/64) and a 4-byte aligned buffer; both are checked
+    before anything is launched."""
+    s = _shape()
+    n = ctypes.c_size_t(1 << 30)
+    st = ctypes.c_void_p(0)
+    call = lambda out, b0, b1: lib.hs2_full_attn_select(ctypes.byref(s), P, P, P, None, None, P, P, P, P, P,
+                                                        ctypes.byref(n), out, b0, b1, st)
+    assert call(P, 3, 3) == hs2.HS2_ERR_INVALID_ARG
+    assert call(P, -1, 2) == hs2.HS2_ERR_INVALID_ARG
+    assert call(P, 0, 33) == hs2.HS2_ERR_INVALID_ARG        # L = 2048: 32 blocks
+    assert call(ctypes.c_void_p(0x1002), 0, 4) == hs2.HS2_ERR_UNSUPPORTED
+    assert hs2.importance_row_stride(s, 32) == 1920 and hs2.importance_row_stride(s, 1) == 64
 
 
 def test_fp8_needs_scales(lib):
@@ -182,6 +198,20 @@ def test_quantize_kv_argument_checks(lib):
     assert lib.hs2_quantize_kv(16, 2, ctypes.c_void_p(0x10008), 256, 128, P, 256, 128, P, st) == \
         hs2.HS2_ERR_UNSUPPORTED
     assert lib.hs2_quantize_kv(16, 2, P, 256, 128, P, 260, 128, P, st) == hs2.HS2_ERR_UNSUPPORTED
+
+
+def test_block_select_longest_sequence(lib):
+    """Block-level selection holds a row's pooled values (L / 64 floats) in
+    64 KiB of shared memory: L = 2^20 passes the size check (and fails on the
+    null index buffer), L = 2^21 is refused before anything is launched."""
+    st = ctypes.c_void_p(0)
+    for L, code in ((1 << 20, hs2.HS2_ERR_INVALID_ARG), (1 << 21, hs2.HS2_ERR_UNSUPPORTED)):
+        s = ctypes.byref(_shape(L=L, Hq=16, Hkv=2, q_tok_stride=16 * 128))
+        assert lib.hs2_block_select(s, P, L, 0, 1, None, P, st) == code
+    s = ctypes.byref(_shape(L=1 << 21, Hq=16, Hkv=2, q_tok_stride=16 * 128))
+    n = ctypes.c_size_t(1 << 40)
+    assert lib.hs2_full_attn_select_blocks(s, P, P, P, None, None, P, P, P, P, P, ctypes.byref(n), st) == \
+        hs2.HS2_ERR_UNSUPPORTED
 
 
 def test_block_select_needs_topk_multiple_of_64(lib):

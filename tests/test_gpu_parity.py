@@ -105,6 +105,43 @@ def test_importance_matches_oracle(L, Hq, Hkv):
     assert worst <= H.IMP_RTOL, worst
 
 
+@pytest.mark.parametrize("L,Hq,Hkv,kv", [(2304, 8, 1, "bf16"), (1536, 16, 2, "bf16"), (1088, 8, 2, "e4m3")])
+def test_importance_mass_conservation_on_gpu(L, Hq, Hkv, kv):
+    """Checking mode (debug flag bit 1): kernel (2) over every visible key
+    j < e_b with the causal mask.  A row then holds, for each key, the
+    probabilities the block's 64 queries of the group's G heads give it, so
+    it sums to 64 * G when the GPU's own LSE normalises every query; the
+    candidate part must equal the normal row bit for bit."""
+    wl = inputs.Workload(f"m{L}", L, Hq, Hkv, 0, seed=19, kv_dtype=kv)
+    xd = H.to_dev(inputs.make_inputs(wl), DEV)
+    shape = H.shape_of(wl, xd)
+    q0, k, v, ks, vs = xd["q_layers"][0], xd["k"], xd["v"], xd.get("k_scale"), xd.get("v_scale")
+    o = torch.empty_like(q0)
+    lse = torch.empty((Hq, L), device=DEV)
+    hs2.hs2_attn_fwd(shape, q0, k, v, ks, vs, o, lse)
+    nb = L // 64
+    full = torch.full((Hkv, nb, L), float("nan"), device=DEV)
+    hs2.hs2_debug_set(H.WAIT_LIMIT_NS, 2)
+    try:
+        hs2.hs2_importance(shape, q0, k, ks, lse, 0, nb, full, L)
+        hs2.hs2_sync()
+    finally:
+        hs2.hs2_debug_set(H.WAIT_LIMIT_NS, 0)
+    normal = H.gpu_importance(shape, xd, lse, 0, nb).cpu().numpy()
+    full = full.cpu().numpy()
+    G = Hq // Hkv
+    worst = 0.0
+    for b in range(nb):
+        _, e_b = orc.block_rows(b, L, 64)
+        n_c = orc.n_candidates(e_b, 128)
+        for g in range(Hkv):
+            row = full[g, b, :e_b].astype(np.float64)
+            assert np.all(np.isfinite(row)) and np.all(row >= 0)
+            worst = max(worst, abs(row.sum() - 64 * G) / (64 * G))
+            assert np.array_equal(full[g, b, :n_c].view(np.uint32), normal[g, b, :n_c].view(np.uint32)), (g, b)
+    assert worst <= 1e-4, worst
+
+
 # ------------------------------------------------------------ kernel (3) --
 
 @pytest.mark.parametrize("L,Hq,Hkv", [(2304, 8, 1), (1536, 8, 2)])
@@ -124,6 +161,45 @@ def test_select_bit_exact_on_exported_importance(L, Hq, Hkv):
             assert cnt[g, b] == wc
             assert np.array_equal(idx[g, b], want), (g, b)
     assert all(H.guards_intact(bb) for bb in r["bases"])
+
+
+@pytest.mark.parametrize("L,Hq,Hkv,strips", [(4096, 8, 2, 5), (2560, 16, 2, 1)])
+def test_select_bit_exact_on_the_rows_the_selection_consumed(L, Hq, Hkv, strips):
+    """hs2_full_attn_select's own export of the importance rows it selected
+    from (a small workspace, so the export spans several strips): the oracle's
+    select on those rows gives the GPU's lists bit for bit, and the rows equal
+    hs2_importance's recompute bit for bit."""
+    wl = _wl(L, Hq, Hkv, n_sparse=0, seed=17)
+    xd = H.to_dev(inputs.make_inputs(wl), DEV)
+    shape = H.shape_of(wl, xd)
+    q0, k, v = xd["q_layers"][0], xd["k"], xd["v"]
+    nb = L // 64
+    b0, b1 = 10, nb - 3
+    S = hs2.importance_row_stride(shape, b1)
+    exp_t = torch.full((Hkv, b1 - b0, S), float("nan"), device=DEV, dtype=torch.float32)
+    row = (L - 128 + 63) // 64 * 64 * 4
+    ws = torch.empty(strips * Hkv * row // 4 + 16, device=DEV, dtype=torch.float32)
+    out = hs2.alloc_outputs(shape, q0, with_workspace=False)
+    hs2.hs2_full_attn_select(shape, q0, k, v, None, None, out["o"], out["lse"], out["idx"], out["cnt"], ws,
+                             importance_out=exp_t, strip=(b0, b1))
+    hs2.hs2_sync()
+    rows = exp_t.cpu().numpy()
+    re = H.gpu_importance(shape, xd, out["lse"], b0, b1).cpu().numpy()
+    idx, cnt = out["idx"].cpu().numpy(), out["cnt"].cpu().numpy()
+    checked = 0
+    for bi, b in enumerate(range(b0, b1)):
+        _, e_b = orc.block_rows(b, L, 64)
+        n_c = orc.n_candidates(e_b, 128)
+        for g in range(Hkv):
+            if n_c <= wl.topk:
+                assert np.isnan(rows[g, bi]).all()       # no importance is computed there
+                continue
+            r_row = rows[g, bi, :n_c]
+            assert np.array_equal(r_row.view(np.uint32), re[g, bi, :n_c].view(np.uint32)), (g, b)
+            want, wc = orc.select(r_row.astype(np.float64), 1024, 128, e_b)
+            assert cnt[g, b] == wc and np.array_equal(idx[g, b], want), (g, b)
+            checked += 1
+    assert checked > 0
 
 
 def _crafted_rows(n, rng):
@@ -427,6 +503,58 @@ def test_fp8_attn_fwd_matches_oracle(L, Hq, Hkv):
     H.bf16_close(o.float().cpu().numpy(), O, "O (fp8 cache)")
     assert np.abs(lse.cpu().numpy() - LSE).max() <= H.LSE_ATOL
     assert H.guards_intact(ob) and H.guards_intact(lb)
+
+
+def test_fp8_q_at_the_edges_of_f16():
+    """With an e4m3 cache Q is rounded bf16 -> f16: exact for magnitudes in
+    [2^-14, 65504], subnormal below.  Rows holding 6e4 (sharp softmax) and
+    rows scaled by 2^-20 (f16 subnormals: flat softmax) still match the
+    oracle on the whole path; a Q value of 1e5 (no f16 value) is reported as
+    HS2_ERR_RANGE by hs2_sync for the full-attention and the sparse kernel."""
+    L, Hq, Hkv = 1536, 8, 2
+    wl = _fp8_wl(L, Hq, Hkv, n_sparse=1, seed=37)
+    x = inputs.make_inputs(wl)
+    rng = np.random.default_rng(3)
+    for q in x["q_layers"]:
+        big = rng.choice(L * Hq, 200, replace=False)
+        tiny = rng.choice(np.setdiff1d(np.arange(L * Hq), big), 200, replace=False)
+        flat = q.view(L * Hq, 128)
+        flat[big, 0] = 6.0e4
+        flat[big, 1] = -6.0e4
+        flat[tiny] = (flat[tiny].float() * 2.0 ** -20).to(torch.bfloat16)
+    xd = H.to_dev(x, DEV)
+    r = H.run_path(wl, xd)
+    D = H.decode(x)
+    O, LSE = orc.dense_attn(D["Q"][0], D["K"], D["V"])
+    H.bf16_close(r["o"].float().cpu().numpy(), O, "O (Q at the f16 edges)")
+    assert (np.abs(r["lse"].cpu().numpy() - LSE) <= H.LSE_ATOL + 1e-6 * np.abs(LSE)).all()
+    nb = L // 64
+    imp = H.gpu_importance(r["shape"], xd, r["lse"], 0, nb).cpu().numpy().astype(np.float64)
+    idx, cnt = r["idx"].cpu().numpy(), r["cnt"].cpu().numpy()
+    ref_sp = np.empty((L, Hq, 128))
+    for b in range(nb):
+        s_b, e_b = orc.block_rows(b, L, 64)
+        for g in range(Hkv):
+            n_c = orc.n_candidates(e_b, 128)
+            want, wc = orc.select(imp[g, b, :n_c], wl.topk, 128, e_b)
+            assert cnt[g, b] == wc and np.array_equal(idx[g, b], want), (g, b)
+            ref_sp[s_b:e_b, g * 4:(g + 1) * 4] = orc.sparse_attn(D["Q"][1], D["K"], D["V"], idx[g, b], wc, b, g, 64)
+    H.bf16_close(r["sparse"][0].float().cpu().numpy(), ref_sp, "sparse (Q at the f16 edges)")
+
+    bad = [q.clone() for q in xd["q_layers"]]
+    for q in bad:
+        q[100, 3, 17] = 1.0e5
+    o = torch.empty_like(bad[0])
+    lse = torch.empty((Hq, L), device=DEV)
+    hs2.hs2_attn_fwd(r["shape"], bad[0], xd["k"], xd["v"], xd["k_scale"], xd["v_scale"], o, lse)
+    with pytest.raises(hs2.Hs2Error) as e:
+        hs2.hs2_sync()
+    assert e.value.code == hs2.HS2_ERR_RANGE
+    hs2.hs2_sparse_attn(r["shape"], bad[1], xd["k"], xd["v"], xd["k_scale"], xd["v_scale"], r["idx"], r["cnt"], o)
+    with pytest.raises(hs2.Hs2Error) as e:
+        hs2.hs2_sync()
+    assert e.value.code == hs2.HS2_ERR_RANGE
+    hs2.hs2_sync()   # the status was cleared
 
 
 @pytest.mark.parametrize("L,Hq,Hkv", [(2304, 8, 1), (1536, 4, 2)])

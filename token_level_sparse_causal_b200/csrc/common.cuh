@@ -167,6 +167,23 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// True when a half of `f16x2` is infinite although the matching half of
+// `bf16x2` (the value it was rounded from) is finite: a bf16 magnitude of
+// 65520 or more has no f16 value.
+__device__ __forceinline__ bool f16_overflowed(uint32_t bf16x2, uint32_t f16x2) {
+  const bool inf_lo = (f16x2 & 0x7FFFu) == 0x7C00u, inf_hi = (f16x2 & 0x7FFF0000u) == 0x7C000000u;
+  const bool fin_lo = (bf16x2 & 0x7F80u) != 0x7F80u, fin_hi = (bf16x2 & 0x7F800000u) != 0x7F800000u;
+  return (inf_lo && fin_lo) || (inf_hi && fin_hi);
+}
+
+// bf16x8_to_f16x8 that also flags a value f16 cannot hold (see f16_overflowed).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8_checked(uint4 v, bool& overflow) {
+  const uint4 h = bf16x8_to_f16x8(v);
+  overflow |= f16_overflowed(v.x, h.x) | f16_overflowed(v.y, h.y) | f16_overflowed(v.z, h.z) |
+              f16_overflowed(v.w, h.w);
+  return h;
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t h;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(hi), "f"(lo));

@@ -176,7 +176,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) sparse_decode_kernel(const Dec
 #pragma unroll
       for (int hlf = 0; hlf < 2; ++hlf) {
         uint32_t w = live ? *reinterpret_cast<const uint32_t*>(qr + 16 * ks + 8 * hlf + 2 * tq) : 0u;
-        if (KV8) w = pack_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+        if (KV8) {
+          const uint32_t h = pack_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+          if (f16_overflowed(w, h)) report(HS2_ERR_RANGE, 399);
+          w = h;
+        }
         qa[ks][hlf] = w;
       }
     }

@@ -66,6 +66,7 @@ constexpr int KVM_BF16 = 0;  // bf16 cache, TMA
 constexpr int KVM_E4M3 = 1;  // e4m3 codes, converted in the kernel
 constexpr int KVM_F16 = 2;   // f16 copy of an e4m3 cache (+ K column scales), TMA
 constexpr uint32_t FLAG_SKIP_LOADS = 1u;
+constexpr uint32_t FLAG_IMP_VISIBLE = 2u;  // hs2_importance over every visible key (checking mode)
 constexpr int MAX_LIST = 4096;
 
 struct FlashParams {
@@ -309,10 +310,12 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       const int pt = threadIdx.x - 64;  // 0..63
       if (mbar_wait(&bars->q_raw, 0, p.limit_ns, abort_flag, 141)) {
         const int nchunks = (has_b ? 2 : 1) * static_cast<int>(TILE_BYTES / 16);
+        bool q_over = false;
         for (int c = pt; c < nchunks; c += 64) {
           const uint32_t a = q_base + c * 16;
-          st_shared_v4(a, bf16x8_to_f16x8(ld_shared_v4(a)));
+          st_shared_v4(a, bf16x8_to_f16x8_checked(ld_shared_v4(a), q_over));
         }
+        if (q_over) report(HS2_ERR_RANGE, 149);
         fence_proxy_async_smem();
         mbar_arrive(&bars->q_full);
         // K/V tiles: 8 threads per 128-byte code row, 16 codes -> two f16 chunks each

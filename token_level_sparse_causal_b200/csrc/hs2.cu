@@ -123,9 +123,30 @@ int sm_count() {
 
 float scale_log2(int d) { return static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d))); }
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per (kernel, device): the attribute is per device, so a
+// process that drives several GPUs sets it on each.
 template <typename K>
 int set_smem(K kernel, uint32_t bytes) {
-  return cuda_ok(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)));
+  struct Done {
+    const void* fn;
+    int dev;
+    uint32_t bytes;
+  };
+  static std::mutex mu;
+  static Done done[256];
+  static int n_done = 0;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HS2_ERR_CUDA;
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done[i].fn == fn && done[i].dev == dev && done[i].bytes >= bytes) return HS2_OK;
+  if (int rc = cuda_ok(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(bytes))))
+    return rc;
+  if (n_done < 256) done[n_done++] = Done{fn, dev, bytes};
+  return HS2_OK;
 }
 
 // ------------------------------------------------------------- launches --
@@ -230,16 +251,13 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
   p.flags = g_flags;
   const unsigned grid = static_cast<unsigned>(p.npairs * s->Hq);
   if (kv8 && dq) {
-    static int attr16 = set_smem(flash_fwd_kernel<KVM_F16>, FL_SMEM_KV8);
-    if (attr16) return attr16;
+    if (int rc_smem = set_smem(flash_fwd_kernel<KVM_F16>, FL_SMEM_KV8)) return rc_smem;
     flash_fwd_kernel<KVM_F16><<<grid, FL_THREADS, FL_SMEM_KV8, st>>>(mq, mk, mv, p);
   } else if (kv8) {
-    static int attr8 = set_smem(flash_fwd_kernel<KVM_E4M3>, FL_SMEM_KV8);
-    if (attr8) return attr8;
+    if (int rc_smem = set_smem(flash_fwd_kernel<KVM_E4M3>, FL_SMEM_KV8)) return rc_smem;
     flash_fwd_kernel<KVM_E4M3><<<grid, FL_THREADS, FL_SMEM_KV8, st>>>(mq, mk, mv, p);
   } else {
-    static int attr = set_smem(flash_fwd_kernel<KVM_BF16>, FL_SMEM_DENSE);
-    if (attr) return attr;
+    if (int rc_smem = set_smem(flash_fwd_kernel<KVM_BF16>, FL_SMEM_DENSE)) return rc_smem;
     flash_fwd_kernel<KVM_BF16><<<grid, FL_THREADS, FL_SMEM_DENSE, st>>>(mq, mk, mv, p);
   }
   return launched();
@@ -293,16 +311,13 @@ int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* 
   const int n_items = p.nb * s->Hkv * p.mpairs;
   const unsigned grid = static_cast<unsigned>(std::min(n_items, sm_count()));
   if (window > 0) {
-    static int attrw = set_smem(sparse_attn_kernel<false, true>, SP_SMEM);
-    if (attrw) return attrw;
+    if (int rc_smem = set_smem(sparse_attn_kernel<false, true>, SP_SMEM)) return rc_smem;
     sparse_attn_kernel<false, true><<<grid, FL_THREADS, SP_SMEM, st>>>(mq, mk, mv, p, n_items);
   } else if (s->kv_dtype == HS2_KV_E4M3) {
-    static int attr8 = set_smem(sparse_attn_kernel<true, false>, SP_SMEM_KV8);
-    if (attr8) return attr8;
+    if (int rc_smem = set_smem(sparse_attn_kernel<true, false>, SP_SMEM_KV8)) return rc_smem;
     sparse_attn_kernel<true, false><<<grid, FL_THREADS, SP_SMEM_KV8, st>>>(mq, mk, mv, p, n_items);
   } else {
-    static int attr = set_smem(sparse_attn_kernel<false, false>, SP_SMEM);
-    if (attr) return attr;
+    if (int rc_smem = set_smem(sparse_attn_kernel<false, false>, SP_SMEM)) return rc_smem;
     sparse_attn_kernel<false, false><<<grid, FL_THREADS, SP_SMEM, st>>>(mq, mk, mv, p, n_items);
   }
   return launched();
@@ -373,12 +388,10 @@ int launch_decode(const hs2_shape* s, const void* q, const int32_t* positions, i
   }
   const dim3 grid(static_cast<unsigned>(pl.splits), static_cast<unsigned>(s->Hkv), static_cast<unsigned>(n));
   if (s->kv_dtype == HS2_KV_E4M3) {
-    static int attr8 = set_smem(sparse_decode_kernel<true>, DecSmem<true>::BYTES);
-    if (attr8) return attr8;
+    if (int rc_smem = set_smem(sparse_decode_kernel<true>, DecSmem<true>::BYTES)) return rc_smem;
     sparse_decode_kernel<true><<<grid, DEC_THREADS, DecSmem<true>::BYTES, st>>>(p);
   } else {
-    static int attr = set_smem(sparse_decode_kernel<false>, DecSmem<false>::BYTES);
-    if (attr) return attr;
+    if (int rc_smem = set_smem(sparse_decode_kernel<false>, DecSmem<false>::BYTES)) return rc_smem;
     sparse_decode_kernel<false><<<grid, DEC_THREADS, DecSmem<false>::BYTES, st>>>(p);
   }
   return launched();
@@ -389,8 +402,7 @@ int n_cand(const hs2_shape* s, int b) { return std::max(0, std::min(s->L, 64 * (
 template <int G, int KVM>
 int launch_importance_g(const CUtensorMap& mq, const CUtensorMap& mk, const ImpParams& p, dim3 grid,
                         cudaStream_t st) {
-  static int attr = set_smem(importance_kernel<G, KVM>, imp_smem_bytes(G));
-  if (attr) return attr;
+  if (int rc_smem = set_smem(importance_kernel<G, KVM>, imp_smem_bytes(G))) return rc_smem;
   importance_kernel<G, KVM><<<grid, IMP_THREADS, imp_smem_bytes(G), st>>>(mq, mk, p);
   return launched();
 }
@@ -398,10 +410,10 @@ int launch_importance_g(const CUtensorMap& mq, const CUtensorMap& mk, const ImpP
 // Kernel (2) for blocks [b0, b1).  dq as in launch_attn_fwd.
 int launch_importance(const hs2_shape* s, const void* q, const void* k, const float* ks, const float* lse, int b0,
                       int b1, float* imp, int64_t row_stride, int skip_le, cudaStream_t st,
-                      const DequantBuf* dq = nullptr) {
+                      const DequantBuf* dq = nullptr, bool visible = false) {
   const bool kv8 = s->kv_dtype == HS2_KV_E4M3;
   const int G = s->Hq / s->Hkv;
-  const int longest = n_cand(s, b1 - 1);
+  const int longest = visible ? std::min(s->L, 64 * b1) : n_cand(s, b1 - 1);
   if (longest <= 0 || longest <= skip_le) return HS2_OK;
   CUtensorMap mq, mk;
   int rc;
@@ -426,6 +438,7 @@ int launch_importance(const hs2_shape* s, const void* q, const void* k, const fl
   p.b0 = b0;
   p.nbs = b1 - b0;
   p.skip_le = skip_le;
+  p.visible = visible ? 1 : 0;
   p.scale_log2 = scale_log2(s->d);
   p.lse = lse;
   p.imp = imp;
@@ -448,6 +461,10 @@ int launch_importance(const hs2_shape* s, const void* q, const void* k, const fl
   }
 }
 
+// Pooled block values of one row live in shared memory: L / 64 * 4 bytes,
+// at most 64 KiB, so block-level selection covers L <= 2^20.
+constexpr uint32_t kBlockSelectSmem = 64u * 1024u;
+
 int launch_select(const hs2_shape* s, const float* imp, int64_t row_stride, int b0, int b1, int32_t* idx,
                   int32_t* cnt, cudaStream_t st, bool blocks = false) {
   SelParams p{};
@@ -466,12 +483,11 @@ int launch_select(const hs2_shape* s, const float* imp, int64_t row_stride, int 
   const unsigned grid = static_cast<unsigned>(s->Hkv * (b1 - b0));
   if (blocks) {
     const uint32_t dyn = static_cast<uint32_t>(s->L / 64) * 4u;  // pooled values of the longest row
-    static int attr = set_smem(block_select_kernel, 64u * 1024u);
-    if (attr) return attr;
+    if (dyn > kBlockSelectSmem) return HS2_ERR_UNSUPPORTED;
+    if (int rc_smem = set_smem(block_select_kernel, kBlockSelectSmem)) return rc_smem;
     block_select_kernel<<<grid, SEL_THREADS, dyn, st>>>(p);
   } else {
-    static int attr = set_smem(topk_select_kernel, sizeof(SelSmem));
-    if (attr) return attr;
+    if (int rc_smem = set_smem(topk_select_kernel, sizeof(SelSmem))) return rc_smem;
     topk_select_kernel<<<grid, SEL_THREADS, sizeof(SelSmem), st>>>(p);
   }
   return launched();
@@ -558,6 +574,7 @@ const char* hs2_strerror(int code) {
     case HS2_ERR_CUDA: return "CUDA error";
     case HS2_ERR_TIMEOUT: return "device wait timed out";
     case HS2_ERR_INDEX: return "index list entry out of range";
+    case HS2_ERR_RANGE: return "input value outside the supported range (Q too large for f16 with an e4m3 cache)";
     default: return "unknown hs2 status";
   }
 }
@@ -635,11 +652,13 @@ int hs2_importance(const hs2_shape* shape, const void* q, const void* k, const f
   if (!q || !lse || !imp) return HS2_ERR_INVALID_ARG;
   const int nb = shape->L / 64;
   if (b0 < 0 || b1 > nb || b0 >= b1) return HS2_ERR_INVALID_ARG;
-  if (row_stride % 4 || row_stride < n_cand(shape, b1 - 1)) return HS2_ERR_INVALID_ARG;
+  const bool visible = (g_flags & FLAG_IMP_VISIBLE) != 0;
+  const int64_t longest = visible ? std::min(shape->L, 64 * b1) : n_cand(shape, b1 - 1);
+  if (row_stride % 4 || row_stride < longest) return HS2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(imp)) return HS2_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(shape->Hkv) * (b1 - b0) > kMaxStripRows) return HS2_ERR_UNSUPPORTED;
   return launch_importance(shape, q, k, k_scale, lse, b0, b1, imp, row_stride, -1,
-                           static_cast<cudaStream_t>(stream));
+                           static_cast<cudaStream_t>(stream), nullptr, visible);
 }
 
 int hs2_topk_select(const hs2_shape* shape, const float* imp, int64_t row_stride, int32_t b0, int32_t b1,
@@ -658,9 +677,15 @@ int hs2_topk_select(const hs2_shape* shape, const float* imp, int64_t row_stride
 
 namespace hs2 {
 namespace {
+// Optional export of the importance rows a full-layer call computed for
+// blocks [b0, b1) (see hs2_full_attn_select in hs2.h).
+struct ImpExport {
+  float* out = nullptr;
+  int b0 = 0, b1 = 0;
+};
 int full_attn_select_impl(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
                           const float* v_scale, void* o, float* lse, int32_t* idx, int32_t* cnt, void* workspace,
-                          size_t* workspace_bytes, void* stream, bool blocks);
+                          size_t* workspace_bytes, void* stream, bool blocks, const ImpExport& ex);
 }  // namespace
 }  // namespace hs2
 
@@ -668,17 +693,29 @@ extern "C" {
 
 int hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
                          const float* v_scale, void* o, float* lse, int32_t* idx, int32_t* cnt, void* workspace,
-                         size_t* workspace_bytes, void* stream) {
+                         size_t* workspace_bytes, float* importance_out, int32_t strip_b0, int32_t strip_b1,
+                         void* stream) {
+  ImpExport ex;
+  if (importance_out) {
+    if (!shape) return HS2_ERR_INVALID_ARG;
+    if (strip_b0 < 0 || strip_b0 >= strip_b1 || shape->block <= 0 || strip_b1 > shape->L / shape->block)
+      return HS2_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(importance_out) & 3u) return HS2_ERR_UNSUPPORTED;
+    ex.out = importance_out;
+    ex.b0 = strip_b0;
+    ex.b1 = strip_b1;
+  }
   return full_attn_select_impl(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, workspace, workspace_bytes, stream,
-                               false);
+                               false, ex);
 }
 
 int hs2_full_attn_select_blocks(const hs2_shape* shape, const void* q, const void* k, const void* v,
                                 const float* k_scale, const float* v_scale, void* o, float* lse, int32_t* idx,
                                 int32_t* cnt, void* workspace, size_t* workspace_bytes, void* stream) {
   if (shape && shape->topk % 64) return HS2_ERR_UNSUPPORTED;
+  if (shape && shape->L > 0 && static_cast<uint32_t>(shape->L / 64) * 4u > kBlockSelectSmem) return HS2_ERR_UNSUPPORTED;
   return full_attn_select_impl(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, workspace, workspace_bytes, stream,
-                               true);
+                               true, ImpExport{});
 }
 
 int hs2_block_select(const hs2_shape* shape, const float* imp, int64_t row_stride, int32_t b0, int32_t b1,
@@ -687,6 +724,7 @@ int hs2_block_select(const hs2_shape* shape, const float* imp, int64_t row_strid
   int rc = check_shape(shape);
   if (rc) return rc;
   if (shape->topk % 64) return HS2_ERR_UNSUPPORTED;
+  if (static_cast<uint32_t>(shape->L / 64) * 4u > kBlockSelectSmem) return HS2_ERR_UNSUPPORTED;
   if (!imp || !idx || !cnt) return HS2_ERR_INVALID_ARG;
   const int nb = shape->L / 64;
   if (b0 < 0 || b1 > nb || b0 >= b1) return HS2_ERR_INVALID_ARG;
@@ -699,9 +737,27 @@ int hs2_block_select(const hs2_shape* shape, const float* imp, int64_t row_strid
 
 namespace hs2 {
 namespace {
+// Copies the rows of strip [sb0, sb1) (row stride `stride` in the workspace)
+// that fall in the export range to the caller's buffer.
+int export_rows(const hs2_shape* s, const float* imp, int sb0, int sb1, int64_t stride, const ImpExport& ex,
+                cudaStream_t st) {
+  const int lo = std::max(sb0, ex.b0), hi = std::min(sb1, ex.b1);
+  if (!ex.out || lo >= hi) return HS2_OK;
+  const int64_t ostride = strip_stride(s, ex.b1 - 1);
+  const size_t width = static_cast<size_t>(std::min(stride, ostride)) * 4u;
+  for (int g = 0; g < s->Hkv; ++g) {
+    float* dst = ex.out + (static_cast<int64_t>(g) * (ex.b1 - ex.b0) + (lo - ex.b0)) * ostride;
+    const float* src = imp + (static_cast<int64_t>(g) * (sb1 - sb0) + (lo - sb0)) * stride;
+    if (cudaMemcpy2DAsync(dst, static_cast<size_t>(ostride) * 4u, src, static_cast<size_t>(stride) * 4u, width,
+                          static_cast<size_t>(hi - lo), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return HS2_ERR_CUDA;
+  }
+  return HS2_OK;
+}
+
 int full_attn_select_impl(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
                           const float* v_scale, void* o, float* lse, int32_t* idx, int32_t* cnt, void* workspace,
-                          size_t* workspace_bytes, void* stream, bool blocks) {
+                          size_t* workspace_bytes, void* stream, bool blocks, const ImpExport& ex) {
   int rc = check_shape(shape);
   if (rc) return rc;
   if (!workspace_bytes) return HS2_ERR_INVALID_ARG;
@@ -746,6 +802,7 @@ int full_attn_select_impl(const hs2_shape* shape, const void* q, const void* k, 
       const int64_t stride = strip_stride(shape, b1 - 1);
       if ((rc = launch_importance(shape, q, k, k_scale, lse, b, b1, imp, stride, shape->topk, st, dq))) return rc;
       if ((rc = launch_select(shape, imp, stride, b, b1, idx, cnt, st, blocks))) return rc;
+      if ((rc = export_rows(shape, imp, b, b1, stride, ex, st))) return rc;
     }
     b = b1;
   }
@@ -762,10 +819,11 @@ int hs2_full_attn_select_static(const hs2_shape* shape, const void* q, const voi
   int rc = check_shape(shape);
   if (rc) return rc;
   if (min_workspace(shape) > kStaticScratchBytes) return HS2_ERR_WORKSPACE;  // before any CUDA call
+  if (!q || !k || !v || !o || !lse || !idx || !cnt) return HS2_ERR_INVALID_ARG;
   void* scratch = nullptr;
   if ((rc = static_scratch(&scratch))) return rc;
   size_t n = kStaticScratchBytes;
-  return hs2_full_attn_select(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, scratch, &n, stream);
+  return hs2_full_attn_select(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, scratch, &n, nullptr, 0, 0, stream);
 }
 
 int hs2_quantize_kv(int32_t L, int32_t Hkv, const void* src, int64_t src_tok_stride, int64_t src_head_stride,

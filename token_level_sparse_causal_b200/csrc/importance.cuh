@@ -34,6 +34,8 @@
 // (chunks of the longest row of the strip) x (Hkv * blocks).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "flash.cuh"
 
@@ -48,6 +50,7 @@ struct ImpParams {
   const float* ksc;
   int64_t kv_tok, kv_head;
   int skip_le;       // rows with |C_b| <= skip_le are not computed (-1: compute all)
+  int visible;       // checking mode: rows over every key j < e_b, causal mask applied
   float scale_log2;  // log2(e) / sqrt(d)
   const float* lse;  // [Hq][L]
   float* imp;
@@ -98,7 +101,7 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
   const int g = y / p.nbs;
   const int b = p.b0 + y % p.nbs;
   const int e_b = min(p.L, 64 * (b + 1));
-  const int n_c = max(0, e_b - p.recent);
+  const int n_c = p.visible ? e_b : max(0, e_b - p.recent);
   const int j0 = static_cast<int>(blockIdx.x) * IMP_CK;
   if (j0 >= n_c || n_c <= p.skip_le) return;  // uniform exit before any allocation
   const int ntiles = (min(IMP_CK, n_c - j0) + 127) / 128;
@@ -210,10 +213,12 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
     if (KV8 && !(p.flags & FLAG_SKIP_LOADS)) {
       const int pt = threadIdx.x - 64;
       if (mbar_wait(&bars->q_raw, 0, p.limit_ns, abort_flag, 241)) {
+        bool q_over = false;
         for (int c = pt; c < static_cast<int>(2 * QHALF / 16); c += 64) {
           const uint32_t a = q_base + c * 16;
-          st_shared_v4(a, bf16x8_to_f16x8(ld_shared_v4(a)));
+          st_shared_v4(a, bf16x8_to_f16x8_checked(ld_shared_v4(a), q_over));
         }
+        if (q_over) report(HS2_ERR_RANGE, 249);
         fence_proxy_async_smem();
         mbar_arrive(&bars->q_full);
         const int rsub = pt >> 3, c8 = pt & 7;
@@ -278,27 +283,48 @@ __global__ void __launch_bounds__(IMP_THREADS, 1)
         tc_fence_before();
         mbar_arrive(&bars->acc_empty[buf]);  // the buffer's data is in registers now
         const float4* nl4 = reinterpret_cast<const float4*>(nlse + sub * NSUB + col0);
+        // MASK (checking mode only, on the tiles that reach the block's own
+        // positions): key j is visible to column n (query 64b + n / G) iff
+        // n >= (j - 64b) * G.
+        auto accumulate = [&](auto mask_tag) {
+          constexpr bool MASK = decltype(mask_tag)::value;
+          const int nmin = MASK ? (j0 + t * 128 + r - 64 * b) * G - (sub * NSUB + col0) : 0;
 #pragma unroll
-        for (int c = 0; c < NLD; ++c) {
+          for (int c = 0; c < NLD; ++c) {
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 nl = nl4[c * 8 + e4];  // broadcast read
-            const uint64_t a01 = f2_fma(f2_pack(__uint_as_float(sr[c][4 * e4]), __uint_as_float(sr[c][4 * e4 + 1])),
-                                        c2t, f2_pack(nl.x, nl.y));
-            const uint64_t a23 = f2_fma(
-                f2_pack(__uint_as_float(sr[c][4 * e4 + 2]), __uint_as_float(sr[c][4 * e4 + 3])), c2t,
-                f2_pack(nl.z, nl.w));
-            // 2 of every 8 columns take the FMA-pipe exponential (exp2_fma3,
-            // relative error 7.5e-5): measured fastest at this share
-            float x0, x1, x2, x3;
-            f2_unpack(a01, x0, x1);
-            f2_unpack(a23, x2, x3);
-            const float y0 = ((e4 & 1) == 0) ? exp2_fma3(x0) : ex2_approx(x0);
-            const float y2 = ((e4 & 1) == 1) ? exp2_fma3(x2) : ex2_approx(x2);
-            acc2[0] = f2_add(acc2[0], f2_pack(y0, ex2_approx(x1)));
-            acc2[1] = f2_add(acc2[1], f2_pack(y2, ex2_approx(x3)));
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 nl = nl4[c * 8 + e4];  // broadcast read
+              const uint64_t a01 = f2_fma(
+                  f2_pack(__uint_as_float(sr[c][4 * e4]), __uint_as_float(sr[c][4 * e4 + 1])), c2t,
+                  f2_pack(nl.x, nl.y));
+              const uint64_t a23 = f2_fma(
+                  f2_pack(__uint_as_float(sr[c][4 * e4 + 2]), __uint_as_float(sr[c][4 * e4 + 3])), c2t,
+                  f2_pack(nl.z, nl.w));
+              // 2 of every 8 columns take the FMA-pipe exponential (exp2_fma3,
+              // relative error 7.5e-5): measured fastest at this share
+              float x0, x1, x2, x3;
+              f2_unpack(a01, x0, x1);
+              f2_unpack(a23, x2, x3);
+              float y0 = ((e4 & 1) == 0) ? exp2_fma3(x0) : ex2_approx(x0);
+              float y1 = ex2_approx(x1);
+              float y2 = ((e4 & 1) == 1) ? exp2_fma3(x2) : ex2_approx(x2);
+              float y3 = ex2_approx(x3);
+              if (MASK) {
+                const int n0 = c * 32 + 4 * e4;
+                y0 = (n0 >= nmin) ? y0 : 0.f;
+                y1 = (n0 + 1 >= nmin) ? y1 : 0.f;
+                y2 = (n0 + 2 >= nmin) ? y2 : 0.f;
+                y3 = (n0 + 3 >= nmin) ? y3 : 0.f;
+              }
+              acc2[0] = f2_add(acc2[0], f2_pack(y0, y1));
+              acc2[1] = f2_add(acc2[1], f2_pack(y2, y3));
+            }
           }
-        }
+        };
+        if (p.visible && j0 + t * 128 + 127 >= 64 * b)
+          accumulate(std::true_type{});
+        else
+          accumulate(std::false_type{});
       }
       if (!ok) break;
       // Groups 2..IMP_GROUPS hand their partial sums to group 1 through a

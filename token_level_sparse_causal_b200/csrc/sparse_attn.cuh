@@ -374,10 +374,12 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
             break;
           }
           const int nchunks = (w.has_b ? 2 : 1) * static_cast<int>(TILE_BYTES / 16);
+          bool q_over = false;
           for (int c = pt; c < nchunks; c += 64) {
             const uint32_t a = q_base + c * 16;
-            st_shared_v4(a, bf16x8_to_f16x8(ld_shared_v4(a)));
+            st_shared_v4(a, bf16x8_to_f16x8_checked(ld_shared_v4(a), q_over));
           }
+          if (q_over) report(HS2_ERR_RANGE, 349);
           fence_proxy_async_smem();
           mbar_arrive(&bars->q_full);
           // ---- K/V tiles: 8 threads per 128-byte code row

@@ -16,7 +16,8 @@ import torch
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhs2.so")
 
-HS2_OK, HS2_ERR_INVALID_ARG, HS2_ERR_UNSUPPORTED, HS2_ERR_WORKSPACE, HS2_ERR_CUDA, HS2_ERR_TIMEOUT, HS2_ERR_INDEX = range(7)
+(HS2_OK, HS2_ERR_INVALID_ARG, HS2_ERR_UNSUPPORTED, HS2_ERR_WORKSPACE, HS2_ERR_CUDA, HS2_ERR_TIMEOUT, HS2_ERR_INDEX,
+ HS2_ERR_RANGE) = range(8)
 HS2_KV_BF16, HS2_KV_E4M3 = 0, 1
 
 EXPORTS = ("hs2_full_attn_select", "hs2_sparse_attn", "hs2_sync", "hs2_attn_fwd", "hs2_importance",
@@ -44,7 +45,7 @@ _lib: Optional[ctypes.CDLL] = None
 _vp, _i32, _i64, _u32, _u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64
 _SIGS = {
     "hs2_full_attn_select": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
-                             ctypes.POINTER(ctypes.c_size_t), _vp],
+                             ctypes.POINTER(ctypes.c_size_t), _vp, _i32, _i32, _vp],
     "hs2_full_attn_select_static": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "hs2_full_attn_select_blocks": [ctypes.POINTER(Hs2Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                     ctypes.POINTER(ctypes.c_size_t), _vp],
@@ -117,15 +118,26 @@ def make_shape(q: torch.Tensor, k: torch.Tensor, topk: int = 1024, recent: int =
 def workspace_bytes(shape: Hs2Shape) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().hs2_full_attn_select(ctypes.byref(shape), None, None, None, None, None, None, None, None, None,
-                                      None, ctypes.byref(n), None), "hs2_full_attn_select(size query)")
+                                      None, ctypes.byref(n), None, 0, 0, None), "hs2_full_attn_select(size query)")
     return int(n.value)
 
 
-def hs2_full_attn_select(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, workspace, stream=None) -> None:
+def importance_row_stride(shape, b1: int) -> int:
+    """Row stride (floats) of hs2_full_attn_select's importance export for the
+    block range ending at b1: max(64, roundup(e_{b1-1} - recent, 64))."""
+    n_c = max(0, min(shape.L, shape.block * b1) - shape.recent)
+    return max(64, (n_c + 63) // 64 * 64)
+
+
+def hs2_full_attn_select(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, workspace, stream=None,
+                         importance_out=None, strip=(0, 0)) -> None:
+    """importance_out: optional fp32 tensor of Hkv * (b1 - b0) * importance_row_stride(shape, b1)
+    elements receiving the importance rows of blocks strip = (b0, b1) that the selection consumed."""
     n = ctypes.c_size_t(workspace.numel() * workspace.element_size())
     _check(lib().hs2_full_attn_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale),
                                       _ptr(o), _ptr(lse), _ptr(idx), _ptr(cnt), _ptr(workspace), ctypes.byref(n),
-                                      _stream(stream)), "hs2_full_attn_select")
+                                      _ptr(importance_out), int(strip[0]), int(strip[1]), _stream(stream)),
+           "hs2_full_attn_select")
 
 
 def hs2_full_attn_select_static(shape, q, k, v, k_scale, v_scale, o, lse, idx, cnt, stream=None) -> None:
