@@ -38,7 +38,13 @@
 // Per key tile j the MMA thread issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1),
 // so while softmax A works on S_A(j+1) the tensor core runs PV_B(j) and
 // S_B(j+1), and vice versa: the two softmax warpgroups take turns and the
-// tensor core always has the other tile's work.
+// tensor core always has the other tile's work.  Only P stands between a
+// softmax phase and the products that follow it: the MMA thread checks that
+// V(j) and K(j + 1) landed before it waits for P; a stage's K is released
+// after both S products of its tile, its V after both P V products; the
+// softmax needs no wait on the previous P V (s_full's commit covers it, as a
+// commit covers every earlier MMA of the thread), and O is signalled only
+// after a tile's last product.
 //
 // Softmax runs in the log2 domain with a lazily updated reference max: O is
 // rescaled only when a row max grows by more than 8 (P stays below 256; the
@@ -98,7 +104,8 @@ struct FlashBars {
   uint64_t q_full;
   uint64_t full_k[FL_STAGES];
   uint64_t full_v[FL_STAGES];
-  uint64_t empty[FL_STAGES];
+  uint64_t empty_k[FL_STAGES];  // the stage's K tile (with an FP8 cache also its column scales) may be replaced
+  uint64_t empty_v[FL_STAGES];  // the stage's V tile may be replaced
   uint64_t s_full[2];  // per query tile
   uint64_t p_ready[2];
   uint64_t o_done[2];
@@ -175,11 +182,12 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
     for (int s = 0; s < FL_STAGES; ++s) {
       mbar_init(&bars->full_k[s], kv_arrivals);
       mbar_init(&bars->full_v[s], kv_arrivals);
-      mbar_init(&bars->empty[s], 1);
+      mbar_init(&bars->empty_k[s], 1);
+      mbar_init(&bars->empty_v[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->s_full[x], 1);
-      mbar_init(&bars->p_ready[x], 128);
+      mbar_init(&bars->p_ready[x], 4);  // one arrival per softmax warp
       mbar_init(&bars->o_done[x], 1);
     }
     mbar_init(&bars->fin, 1);
@@ -209,22 +217,27 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       }
       if (!CONV) {
         int last = -1;
+        // A stage's K is replaced once both S products of its tile executed,
+        // its V once both P V products did (with an FP8 cache the K column
+        // scales are read by the softmax of the tile, so K goes with V).
         for (int j = 0; j < n; ++j) {
-          const int u = j;  // position in this CTA's key-tile stream
-          const int s = u % FL_STAGES;
-          if (u >= FL_STAGES &&
-              !mbar_wait(&bars->empty[s], ((u / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 101))
-            break;
+          const int s = j % FL_STAGES;
+          const uint32_t par = ((j / FL_STAGES) - 1) & 1;
+          if (j >= FL_STAGES && !mbar_wait(&bars->empty_k[s], par, p.limit_ns, abort_flag, 101)) break;
           uint8_t* kd = smem + FL_KV_OFF + s * 2 * TILE_BYTES;
           mbar_arrive_expect_tx(&bars->full_k[s], TILE_BYTES + (KV8 ? 512u : 0u));
           if (KV8) bulk_load(ksc_s + s * 128, p.kcol + static_cast<int64_t>(g) * p.kcol_stride + j * 128, 512u,
                              &bars->full_k[s]);
           tma_load_3d(kd, &tmK, &bars->full_k[s], 0, g, j * 128);
           tma_load_3d(kd + HALF_BYTES, &tmK, &bars->full_k[s], 64, g, j * 128);
+          if (j >= FL_STAGES && !mbar_wait(&bars->empty_v[s], par, p.limit_ns, abort_flag, 105)) {
+            wait_done(&bars->full_k[s], (j / FL_STAGES) & 1, p.limit_ns, 106);  // K(j) in flight
+            break;
+          }
           mbar_arrive_expect_tx(&bars->full_v[s], TILE_BYTES);
           tma_load_3d(kd + TILE_BYTES, &tmV, &bars->full_v[s], 0, g, j * 128);
           tma_load_3d(kd + TILE_BYTES + HALF_BYTES, &tmV, &bars->full_v[s], 64, g, j * 128);
-          last = u;
+          last = j;
         }
         // Never leave a TMA write in flight into memory the CTA gives back.
         for (int u = max(0, last - FL_STAGES + 1); u <= last; ++u) {
@@ -258,7 +271,10 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bdesc, KV8 ? IDESC_PV_F16 : IDESC_PV,
                   (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars->o_done[x]);
+        // O is final after the tile's last product (earlier products are
+        // known complete through s_full: a commit covers every MMA issued
+        // before it)
+        if (j == nx[x] - 1) umma_commit(&bars->o_done[x]);
       };
       bool ok = mbar_wait(&bars->q_full, 0, p.limit_ns, abort_flag, 111);
       if (ok) ok = mbar_wait(&bars->full_k[0], 0, p.limit_ns, abort_flag, 112);
@@ -266,40 +282,37 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         tc_fence_after();
         for (int x = 0; x < 2; ++x)
           if (nx[x] > 0) issue_s(x, 0);
+        if (!KV8) umma_commit(&bars->empty_k[0]);  // K(0) multiplied by both query tiles
       }
       for (int j = 0; j < n && ok; ++j) {
         const int u = j;
         const int s = u % FL_STAGES;
-        bool v_ready = false, k_next = false;
+        // V(j) and K(j + 1) normally landed long ago: check them before
+        // blocking on the softmax, so nothing but P stands between its
+        // arrival and the products
+        if (!mbar_wait(&bars->full_v[s], (u / FL_STAGES) & 1, p.limit_ns, abort_flag, 114)) break;
+        if (j + 1 < n &&
+            !mbar_wait(&bars->full_k[(u + 1) % FL_STAGES], ((u + 1) / FL_STAGES) & 1, p.limit_ns, abort_flag, 115))
+          break;
         for (int x = 0; x < 2 && ok; ++x) {
           if (j >= nx[x]) continue;
           if (!mbar_wait(&bars->p_ready[x], j & 1, p.limit_ns, abort_flag, 113)) {
             ok = false;
             break;
           }
-          if (!v_ready) {
-            if (!mbar_wait(&bars->full_v[s], (u / FL_STAGES) & 1, p.limit_ns, abort_flag, 114)) {
-              ok = false;
-              break;
-            }
-            v_ready = true;
-          }
           tc_fence_after();
           issue_pv(x, j);
-          if (j + 1 < nx[x]) {
-            if (!k_next) {
-              const int s1 = (u + 1) % FL_STAGES;
-              if (!mbar_wait(&bars->full_k[s1], ((u + 1) / FL_STAGES) & 1, p.limit_ns, abort_flag, 115)) {
-                ok = false;
-                break;
-              }
-              k_next = true;
-              tc_fence_after();
-            }
-            issue_s(x, j + 1);
-          }
+          if (j + 1 < nx[x]) issue_s(x, j + 1);
         }
-        if (ok) umma_commit(&bars->empty[s]);
+        if (ok) {
+          // V(j) is read by no later product; K(j + 1) neither, once both S
+          // products of tile j + 1 are queued
+          umma_commit(&bars->empty_v[s]);
+          if (KV8)
+            umma_commit(&bars->empty_k[s]);
+          else if (j + 1 < n)
+            umma_commit(&bars->empty_k[(u + 1) % FL_STAGES]);
+        }
       }
       umma_commit(&bars->fin);
       wait_done(&bars->fin, 0, p.limit_ns, 116);
@@ -325,7 +338,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         for (int j = 0; j < (CONV ? n : 0); ++j) {  // KVM_F16: K/V tiles come by TMA
           const int s = j % FL_STAGES;
           if (j >= FL_STAGES &&
-              !mbar_wait(&bars->empty[s], ((j / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 142))
+              (!mbar_wait(&bars->empty_k[s], ((j / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 142) ||
+               !mbar_wait(&bars->empty_v[s], ((j / FL_STAGES) - 1) & 1, p.limit_ns, abort_flag, 143)))
             break;
           const uint32_t kd = kv_base + s * 2 * TILE_BYTES;
 #pragma unroll 1
@@ -424,18 +438,17 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         for (int c = 0; c < 128; ++c)
           if (c > r) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
       }
-      // ---- row max: 4 independent chains of 3-input max
-      float mx4[4];
+      // ---- row max: 8 independent chains of 3-input max over 16 values each
+      float mx8[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) mx4[q] = __uint_as_float(sr[q][0]);
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t* v = &sr[q >> 1][(q & 1) * 16];
+        float m = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-#pragma unroll
-        for (int e = 0; e < 15; ++e)
-          mx4[q] = fmax3(mx4[q], __uint_as_float(sr[q][1 + 2 * e]), __uint_as_float(sr[q][2 + 2 * e]));
-        mx4[q] = fmaxf(mx4[q], __uint_as_float(sr[q][31]));
+        for (int e = 0; e < 6; ++e) m = fmax3(m, __uint_as_float(v[3 + 2 * e]), __uint_as_float(v[4 + 2 * e]));
+        mx8[q] = fmaxf(m, __uint_as_float(v[15]));
       }
-      const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
       const float m_new = fmaxf(m_used, mx * sc);
       float alpha = 1.f;
       const bool resc = m_new > m_used + 8.f;
@@ -470,13 +483,9 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
         f2_unpack(sum2[1], b0, b1);
         l += (a0 + a1) + (b0 + b1);
       }
-      // ---- O rescale (needs PV(j-1) complete)
+      // ---- O rescale: P V(j - 1) completed before S(j) (it was issued
+      // first by the same thread, and s_full's commit covers it)
       if (t > 0) {
-        if (!warp_wait(&bars->o_done[x], (t - 1) & 1, p.limit_ns, abort_flag, 132)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
@@ -492,13 +501,14 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_ready[x]);
+      __syncwarp();  // one arrival per warp, once all its lanes' stores completed
+      if (lane == 0) mbar_arrive(&bars->p_ready[x]);
     }
     // ---- epilogue
     const bool row_live = i_row < p.L && (x == 0 || has_b);  // a last dense tile may hang past L
     __nv_bfloat16* orow = p.o + static_cast<int64_t>(i_row) * p.o_tok + static_cast<int64_t>(hh) * p.o_head;
     const int nT = nX;  // key tiles of this query tile
-    if (ok && nT > 0 && warp_wait(&bars->o_done[x], (nT - 1) & 1, p.limit_ns, abort_flag, 133)) {
+    if (ok && nT > 0 && warp_wait(&bars->o_done[x], 0, p.limit_ns, abort_flag, 133)) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
