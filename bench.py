@@ -75,7 +75,7 @@ def algorithmic_work(wl) -> dict:
 
 
 FA_SOURCES = ("token_level_sparse_causal_b200/csrc/flash.cuh", "token_level_sparse_causal_b200/csrc/common.cuh")
-FA_TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "flash_fwd_dense_dram_L131072.md")
+FA_TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "flash_fwd_dram_c3.json")
 
 
 def kernel_source_hash(paths=FA_SOURCES) -> str:
@@ -88,21 +88,20 @@ def kernel_source_hash(paths=FA_SOURCES) -> str:
 
 
 def recorded_traffic(workload: str, profile=FA_TRAFFIC_PROFILE):
-    """DRAM bytes per launch of kernel (1) from the committed ncu summary, or
-    None when the kernel sources changed since those counters were taken or
-    the summary covers another workload."""
+    """DRAM bytes per full-size launch of kernel (1), from the committed record
+    of an ncu capture (a JSON sidecar), or None when the kernel sources changed
+    since those counters were taken or the record covers another workload."""
     if not os.path.exists(profile):
         return None
-    fields = {}
-    for line in open(profile):
-        if ":" in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(":", 1)
-            fields[k.strip()] = v.strip()
-    if fields.get("kernel_source_sha256_16") != kernel_source_hash() or fields.get("workload") != workload:
+    try:
+        rec = json.load(open(profile))
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_source_sha256_16") != kernel_source_hash() or rec.get("workload") != workload:
         return None
     try:
-        return float(fields["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
+        return float(rec["dram_bytes_per_launch"])
+    except (KeyError, TypeError, ValueError):
         return None
 
 
@@ -626,7 +625,9 @@ def run_stage(args, wl):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     hq, hkv = (int(t) for t in args.heads.split("/")) if args.heads else (wl.Hq, wl.Hkv)
-    my = wl.scaled(name=f"{wl.name}_stage_h{hq}x{hkv}", Hq=hq, Hkv=hkv, n_sparse=0)
+    L = args.seq or wl.L
+    my = wl.scaled(name=f"{wl.name}_stage_h{hq}x{hkv}" + (f"_L{L}" if args.seq else ""), Hq=hq, Hkv=hkv, n_sparse=0,
+                   L=L)
     x = inputs.make_inputs(my, device=dev, with_needles=bool(my.needles))
     q0, k, v = x["q_layers"][0], x["k"], x["v"]
     ks, vs = x.get("k_scale"), x.get("v_scale")
@@ -695,6 +696,7 @@ def main(argv=None):
     ap.add_argument("--stage", choices=["select", "importance", "fa", "sparse"],
                     help="time one stage alone (1 GPU) and print its line")
     ap.add_argument("--heads", help="with --stage: query/KV heads of the reduced copy, e.g. 16/8")
+    ap.add_argument("--seq", type=int, help="with --stage: sequence length of the reduced copy (default: the workload's)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "cuda":
         ap.error("--warmup must be >= 3")

@@ -2,6 +2,7 @@
 committed kernel (1) DRAM traffic is reported only for the workload and the
 kernel sources it was captured on, and each workload's line names its own
 input recipe."""
+import json
 import os
 
 import bench
@@ -9,30 +10,31 @@ from token_level_sparse_causal_b200 import inputs
 
 
 def test_recorded_traffic_only_for_its_own_workload_and_sources(tmp_path):
-    good = tmp_path / "dram.md"
-    good.write_text("# capture\n\n"
-                    "- workload: c3_L131072_h64x8_gmm\n"
-                    "- dram_bytes_per_launch: 12345\n"
-                    f"- kernel_source_sha256_16: {bench.kernel_source_hash()}\n")
+    good = tmp_path / "dram.json"
+    good.write_text(json.dumps({"workload": "c3_L131072_h64x8_gmm", "dram_bytes_per_launch": 12345,
+                                "kernel_source_sha256_16": bench.kernel_source_hash()}))
     assert bench.recorded_traffic("c3_L131072_h64x8_gmm", str(good)) == 12345.0
     assert bench.recorded_traffic("c4_L262144_h64x8_chains", str(good)) is None
-    stale = tmp_path / "stale.md"
-    stale.write_text("- workload: c3_L131072_h64x8_gmm\n- dram_bytes_per_launch: 12345\n"
-                     "- kernel_source_sha256_16: 0000000000000000\n")
+    stale = tmp_path / "stale.json"
+    stale.write_text(json.dumps({"workload": "c3_L131072_h64x8_gmm", "dram_bytes_per_launch": 12345,
+                                 "kernel_source_sha256_16": "0000000000000000"}))
     assert bench.recorded_traffic("c3_L131072_h64x8_gmm", str(stale)) is None
-    assert bench.recorded_traffic("c3_L131072_h64x8_gmm", str(tmp_path / "missing.md")) is None
+    assert bench.recorded_traffic("c3_L131072_h64x8_gmm", str(tmp_path / "missing.json")) is None
+    bad = tmp_path / "bad.json"
+    bad.write_text("not json")
+    assert bench.recorded_traffic("c3_L131072_h64x8_gmm", str(bad)) is None
 
 
-def test_committed_traffic_summary_is_well_formed():
-    """The committed summary names its workload and a per-launch byte count
-    (whether its hash is current depends on the kernel sources)."""
-    fields = {}
-    for line in open(bench.FA_TRAFFIC_PROFILE):
-        if line.strip().startswith("- ") and ":" in line:
-            k, v = line.strip()[2:].split(":", 1)
-            fields[k.strip()] = v.strip()
-    assert fields["workload"] == inputs.WORKLOADS["c3"].name
-    assert int(fields["dram_bytes_per_launch"]) == int(fields["dram_read_bytes"]) + int(fields["dram_write_bytes"])
+def test_committed_traffic_record_is_well_formed():
+    """The committed record names its workload, the reduced-head copy it was
+    measured on and the scale to a full launch (whether its hash is current
+    depends on the kernel sources)."""
+    if not os.path.exists(bench.FA_TRAFFIC_PROFILE):
+        return
+    rec = json.load(open(bench.FA_TRAFFIC_PROFILE))
+    assert rec["workload"] == inputs.WORKLOADS["c3"].name
+    measured = rec["measured"]["dram_read_bytes"] + rec["measured"]["dram_write_bytes"]
+    assert rec["dram_bytes_per_launch"] == measured * rec["scale_to_full_launch"]
 
 
 def test_data_recipe_names_each_workloads_inputs():
