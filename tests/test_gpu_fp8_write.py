@@ -64,3 +64,28 @@ def test_matches_the_generators_fp8_cache_on_the_1m_workload_rows():
     assert torch.equal(dst, q8["k"]) and torch.equal(scale, q8["k_scale"])   # same bytes as the torch path
     rows = np.random.default_rng(0).integers(0, 65536, 64)
     _check(x["k"][rows].cpu(), dst[rows], scale[rows])
+
+
+def test_every_bf16_value_under_many_scales():
+    """All finite bf16 magnitudes from 2^-20 to 2^15 (both signs), each row
+    completed by an amax that sets one of 41 scales: the codes stay bit-exact
+    wherever x / scale lands, on and next to every e4m3 rounding midpoint."""
+    u = np.arange(0x3580, 0x4700, dtype=np.uint32)            # 2^-20 .. 2^15 as bf16 bit patterns
+    vals = torch.from_numpy((u << 16).view(np.float32)).to(torch.bfloat16)
+    vals = torch.cat([vals, -vals])
+    n = vals.numel() // 127 * 127
+    rows = vals[:n].view(-1, 127)
+    out_rows = []
+    for i, amax in enumerate(np.geomspace(2.0 ** -3, 2.0 ** 16, 41)):
+        a = torch.tensor([amax], dtype=torch.float32).to(torch.bfloat16)
+        r = rows[(torch.arange(rows.shape[0]) % 41) == i]
+        r = r.float().clamp(-float(a), float(a)).to(torch.bfloat16)
+        out_rows.append(torch.cat([r, a.expand(r.shape[0], 1)], dim=1))
+    x = torch.cat(out_rows).view(-1, 1, 128)
+    xd = x.to(DEV)
+    dst = torch.empty(x.shape, dtype=torch.uint8, device=DEV)
+    scale = torch.empty(x.shape[:2], device=DEV)
+    hs2.hs2_quantize_kv(xd, dst, scale)
+    hs2.hs2_sync()
+    _check(x, dst, scale)
+

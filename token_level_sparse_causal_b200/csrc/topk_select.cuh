@@ -482,10 +482,12 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const SelPa
 // replaces; HySparse2 architecture summary, block-selection paragraph): each
 // candidate row is pooled into 64-key blocks, the top topk/64 blocks by pooled
 // importance are kept (ties to the lower block) and expanded to positions.
-// The pooled sum of a block is defined in a fixed fp32 order: 16 lanes each
-// add 4 consecutive values left to right, then a butterfly over the 16 lanes
-// (l ^ 8, ^ 4, ^ 2, ^ 1); every step is commutative, so all lanes hold the
-// same bits.  One 512-thread CTA per row; pooled values live in shared memory.
+// A block's pooled sum is taken in fp32: 16 lanes each add 4 consecutive
+// values left to right, then a butterfly over the 16 lanes (l ^ 8, ^ 4, ^ 2,
+// ^ 1); every step is commutative, so all lanes hold the same bits.  Blocks
+// whose exact sums differ by less than the rounding of a 64-term fp32 sum
+// may rank either way.  One 512-thread CTA per row; pooled values live in
+// shared memory.
 __global__ void __launch_bounds__(SEL_THREADS) block_select_kernel(const SelParams p) {
   extern __shared__ float pooled[];  // [n_blk]
   __shared__ uint32_t hist[2048];
