@@ -315,10 +315,10 @@ int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* 
     sparse_attn_kernel<false, true><<<grid, FL_THREADS, SP_SMEM, st>>>(mq, mk, mv, p, n_items);
   } else if (s->kv_dtype == HS2_KV_E4M3) {
     if (int rc_smem = set_smem(sparse_attn_kernel<true, false>, SP_SMEM_KV8)) return rc_smem;
-    sparse_attn_kernel<true, false><<<grid, FL_THREADS, SP_SMEM_KV8, st>>>(mq, mk, mv, p, n_items);
+    sparse_attn_kernel<true, false><<<grid, sp_threads(true, false), SP_SMEM_KV8, st>>>(mq, mk, mv, p, n_items);
   } else {
     if (int rc_smem = set_smem(sparse_attn_kernel<false, false>, SP_SMEM)) return rc_smem;
-    sparse_attn_kernel<false, false><<<grid, FL_THREADS, SP_SMEM, st>>>(mq, mk, mv, p, n_items);
+    sparse_attn_kernel<false, false><<<grid, sp_threads(false, false), SP_SMEM, st>>>(mq, mk, mv, p, n_items);
   }
   return launched();
 }

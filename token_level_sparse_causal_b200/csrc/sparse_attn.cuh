@@ -29,12 +29,14 @@
 //   * the first P V of an item waits only for the previous epilogue of the
 //     same M tile to have read O (o_free); its S products do not wait.
 //
-// Roles (12 warps), as in flash_fwd_kernel: warp 1 issues every MMA, warps
-// 4-7 / 8-11 run the softmax and epilogue of M tile A / B; with a bf16 cache
-// warps 0, 2 and 3 load the lists, gather K/V and (one thread) load Q; with an
-// FP8 cache warp 0 loads Q by TMA and warps 2-3 convert it and gather and
-// convert the K/V codes to f16; in window mode warp 0 loads Q and whole K/V
-// tiles by TMA.  Every wait is bounded; a wait that runs out
+// Roles, as in flash_fwd_kernel: warp 1 issues every MMA, warps 4-7 / 8-11
+// run the softmax and epilogue of M tile A / B; with a bf16 cache warps 0, 2,
+// 3 and 12-15 load the lists, gather K/V and (one thread) load Q; with an FP8
+// cache warp 0 loads Q by TMA and warps 2, 3, 12 and 13 convert it and gather
+// and convert the K/V codes to f16; in window mode (12 warps) warp 0 loads Q
+// and whole K/V tiles by TMA.  The list modes run 16 warps with registers
+// moved to the softmax warpgroups (the gather's issue rate was the critical
+// path with 3 gather warps).  Every wait is bounded; a wait that runs out
 // records HS2_ERR_TIMEOUT and the CTA winds down.
 #pragma once
 
@@ -60,6 +62,17 @@ struct SparseBars {
   int abort;
 };
 static_assert(sizeof(SparseBars) <= 256, "barriers fit their slot");
+
+// The list modes run 16 warps: the bf16 gather uses 7 of them (0, 2, 3,
+// 12-15), the FP8 converter 4 (2, 3, 12, 13), with registers moved from the
+// copy/MMA warpgroups (0 and 3) to the two softmax warpgroups:
+// 2 x 128 x SP_REG_COPY + 256 x SP_REG_SOFTMAX = 65536 = 512 x 128, the
+// registers the CTA is launched with.  The window mode keeps 12 warps.
+constexpr int SP_THREADS_LIST = 512;
+constexpr uint32_t SP_REG_COPY = 80, SP_REG_SOFTMAX = 176;  // 56 / 200 and 88, 96 measured slower
+static_assert(2 * 128 * SP_REG_COPY + 256 * SP_REG_SOFTMAX <= SP_THREADS_LIST * (65536 / SP_THREADS_LIST),
+              "register split within the launch's registers");
+__host__ __device__ constexpr int sp_threads(bool kv8, bool win) { return !win ? SP_THREADS_LIST : FL_THREADS; }
 
 constexpr uint32_t SP_POS_OFF = FL_POS_OFF;                      // int [2][MAX_LIST]
 constexpr uint32_t SP_KSC_OFF = SP_POS_OFF + 2 * MAX_LIST * 4;   // KV8: [stage][128]
@@ -103,7 +116,7 @@ __device__ __forceinline__ SpItem sparse_item(const FlashParams& p, int it, int 
 }
 
 template <bool KV8, bool WIN>
-__global__ void __launch_bounds__(FL_THREADS, 1)
+__global__ void __launch_bounds__(sp_threads(KV8, WIN), 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const FlashParams p, int n_items) {
   static_assert(!(KV8 && WIN), "the window mode reads a bf16 cache");
@@ -118,12 +131,13 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
   volatile int* abort_flag = &bars->abort;
   const int first = blockIdx.x, step = gridDim.x;
   // loader threads: warps 2-3 with an FP8 cache (warp 0 then only loads Q);
-  // warps 0, 2, 3 with bf16, warp 0's lane 0 also loading Q
-  constexpr int NLD = KV8 ? 64 : 96;
+  // warps 0, 2, 3 and 12-15 with bf16 lists, warp 0's lane 0 also loading Q
+  constexpr bool SPLIT = !WIN;  // 16 warps, registers moved to the softmax
+  constexpr int NLD = KV8 ? 128 : (WIN ? 96 : 224);
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_raw, 1);
-    mbar_init(&bars->q_full, KV8 ? 64u : 1u);
+    mbar_init(&bars->q_full, KV8 ? static_cast<uint32_t>(NLD) : 1u);
     mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < FL_STAGES; ++s) {
       mbar_init(&bars->full_k[s], WIN ? 1 : NLD);
@@ -150,7 +164,10 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_slot;
-
+  // warpgroup index, visibly uniform for the compiler
+  const int wgi = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x) / 128, 0);
+  if (wgi == 0 || wgi == 3) {
+  if (SPLIT) reg_release<SP_REG_COPY>();
   if ((KV8 || WIN) && warp == 0) {
     // ============================ Q by TMA (and, in window mode, K/V tiles)
     if (lane == 0 && !(p.flags & FLAG_SKIP_LOADS)) {
@@ -301,10 +318,12 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       umma_commit(&bars->fin);
       wait_done(&bars->fin, 0, p.limit_ns, 317);
     }
-  } else if (!WIN && (warp == 0 || warp == 2 || warp == 3)) {
+  } else if (!WIN && (KV8 ? (warp == 2 || warp == 3 || warp == 12 || warp == 13)
+                          : (warp == 0 || warp == 2 || warp == 3 || warp >= 12))) {
     // ===================================== lists and K/V (gather / convert)
     if (!(p.flags & FLAG_SKIP_LOADS)) {
-      const int pt = KV8 ? threadIdx.x - 64 : (warp == 0 ? lane : threadIdx.x - 32);  // 0 .. NLD-1
+      const int pt = KV8 ? (warp < 4 ? threadIdx.x - 64 : threadIdx.x - 320)
+                         : (warp == 0 ? lane : (warp < 4 ? threadIdx.x - 32 : threadIdx.x - 288));  // 0 .. NLD-1
       const bool q_thread = !KV8 && warp == 0 && lane == 0;
       if (q_thread) tma_prefetch_desc(&tmQ);
       int ii = 0, u0 = 0, qi = 0, loaded = 0;
@@ -375,14 +394,16 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
           }
           const int nchunks = (w.has_b ? 2 : 1) * static_cast<int>(TILE_BYTES / 16);
           bool q_over = false;
-          for (int c = pt; c < nchunks; c += 64) {
+          for (int c = pt; c < nchunks; c += NLD) {
             const uint32_t a = q_base + c * 16;
             st_shared_v4(a, bf16x8_to_f16x8_checked(ld_shared_v4(a), q_over));
           }
           if (q_over) report(HS2_ERR_RANGE, 349);
           fence_proxy_async_smem();
           mbar_arrive(&bars->q_full);
-          // ---- K/V tiles: 8 threads per 128-byte code row
+          // ---- K/V tiles: 8 threads per 128-byte code row, RPT rows each
+          constexpr int RSTEP = NLD / 8, RPT = 128 / RSTEP;
+          static_assert(!KV8 || RSTEP * RPT == 128, "converter rows cover the tile");
           const int rsub = pt >> 3, c8 = pt & 7;
           const uint8_t* kb8 = p.k8 + static_cast<int64_t>(w.g) * p.kv_head + c8 * 16;
           const uint8_t* vb8 = p.v8 + static_cast<int64_t>(w.g) * p.kv_head + c8 * 16;
@@ -400,11 +421,11 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
               const uint8_t* base8 = half ? vb8 : kb8;
               const float* scale = half ? p.vsc : p.ksc;
               // every row's codes and scale in flight before any is converted
-              uint4 raw[16];
-              float sgv[16];
+              uint4 raw[RPT];
+              float sgv[RPT];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int pj = pos_s[j * 128 + rsub + 8 * i];
+              for (int i = 0; i < RPT; ++i) {
+                const int pj = pos_s[j * 128 + rsub + RSTEP * i];
                 raw[i] = make_uint4(0, 0, 0, 0);
                 sgv[i] = 0.f;
                 if (pj >= 0) {
@@ -413,8 +434,8 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
                 }
               }
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int r = rsub + 8 * i;
+              for (int i = 0; i < RPT; ++i) {
+                const int r = rsub + RSTEP * i;
                 const float sg = sgv[i];
                 const uint32_t wd[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
                 uint32_t f[8];
@@ -489,7 +510,9 @@ __global__ void __launch_bounds__(FL_THREADS, 1)
       cp_async_wait<0>();
       if (q_thread && loaded > 0) wait_done(&bars->q_full, (loaded - 1) & 1, p.limit_ns, 302);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    if (SPLIT) reg_acquire<SP_REG_SOFTMAX>();
     // ============================================ softmax / rescale / epilogue
     const int x = (warp >= 8) ? 1 : 0;  // M tile of this warpgroup
     const int r = threadIdx.x - 128 - 128 * x;
