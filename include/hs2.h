@@ -323,7 +323,11 @@ const char* hs2_strerror(int code);
  * over the candidates C_b (row_stride must then be at least e_{b1-1}): such
  * a row sums to 64 * G (every query's probabilities sum to one), which a test
  * checks; its first |C_b| entries equal the normal row's.  hs2_full_attn_select
- * ignores bit 1.  Flags are 0 in normal use.
+ * ignores bit 1.  Bit 2 runs the full layer's attention (hs2_attn_fwd and
+ * inside hs2_full_attn_select) on clusters of two CTAs that share every
+ * product (tcgen05 cta_group::2) when the cache is bf16 or its f16 layer copy
+ * is in the workspace: the results are bit for bit those of the default
+ * kernel.  Flags are 0 in normal use.
  */
 int hs2_debug_set(uint64_t wait_limit_ns, uint32_t flags);
 

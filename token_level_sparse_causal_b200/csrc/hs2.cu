@@ -18,6 +18,7 @@
 #include "../../include/hs2.h"
 #include "common.cuh"
 #include "flash.cuh"
+#include "flash2.cuh"
 #include "sparse_attn.cuh"
 #include "importance.cuh"
 #include "topk_select.cuh"
@@ -249,6 +250,25 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
   p.lse = lse;
   p.limit_ns = g_wait_limit_ns;
   p.flags = g_flags;
+  if ((g_flags & FLAG_FA_CTA_PAIRS) && p.G % 2 == 0 && (!kv8 || dq)) {
+    // CTA pairs: two heads of a group per cluster (check_shape admits G = 2,
+    // 4, 8), K tiles loaded as 64-key halves
+    CUtensorMap mk64;
+    if (!kv8) {
+      if ((rc = make_map(&mk64, k, s->L, s->Hkv, s->kv_tok_stride, s->kv_head_stride, 1, 64))) return rc;
+    } else {
+      if ((rc = make_map(&mk64, dq->kf, s->L, s->Hkv, int64_t(s->Hkv) * HD, HD, 1, 64))) return rc;
+    }
+    const unsigned grid2 = static_cast<unsigned>(p.npairs * s->Hq);
+    if (kv8) {
+      if (int rc_smem = set_smem(flash2_fwd_kernel<KVM_F16>, F2_SMEM)) return rc_smem;
+      flash2_fwd_kernel<KVM_F16><<<grid2, FL_THREADS, F2_SMEM, st>>>(mq, mk64, mv, p);
+    } else {
+      if (int rc_smem = set_smem(flash2_fwd_kernel<KVM_BF16>, F2_SMEM)) return rc_smem;
+      flash2_fwd_kernel<KVM_BF16><<<grid2, FL_THREADS, F2_SMEM, st>>>(mq, mk64, mv, p);
+    }
+    return launched();
+  }
   const unsigned grid = static_cast<unsigned>(p.npairs * s->Hq);
   if (kv8 && dq) {
     if (int rc_smem = set_smem(flash_fwd_kernel<KVM_F16>, FL_SMEM_KV8)) return rc_smem;
