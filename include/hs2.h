@@ -327,7 +327,13 @@ const char* hs2_strerror(int code);
  * inside hs2_full_attn_select) on clusters of two CTAs that share every
  * product (tcgen05 cta_group::2) when the cache is bf16 or its f16 layer copy
  * is in the workspace: the results are bit for bit those of the default
- * kernel.  Flags are 0 in normal use.
+ * kernel.  Bit 3 makes every TMA descriptor encoding fail as a driver error
+ * would: calls that encode one return HS2_ERR_CUDA before launching anything
+ * (host-side fault injection for tests).  Flags are 0 in normal use.
+ *
+ * Each kernel launch (and each hs2_full_attn_select call) is wrapped in an
+ * NVTX range named after it ("hs2 attn_fwd (kernel 1)", ...), which
+ * profilers can use to attribute and filter launches.
  */
 int hs2_debug_set(uint64_t wait_limit_ns, uint32_t flags);
 

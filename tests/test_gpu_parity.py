@@ -679,6 +679,48 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     H.bf16_close(o.float().cpu().numpy(), O, "O after timeout")
 
 
+def test_host_tensor_map_failure_returns_before_any_launch():
+    """Host-side fault injection (hs2_debug_set bit 3): every TMA descriptor
+    encoding fails as a driver error would.  Each call returns HS2_ERR_CUDA
+    without launching a kernel or touching its outputs, and once the hook is
+    cleared the same calls work."""
+    wl = _wl(1024, 8, 2, seed=31)
+    x = inputs.make_inputs(wl)
+    xd = H.to_dev(x, DEV)
+    r = H.run_path(wl, xd)  # lists for the sparse call
+    q0, k, v = xd["q_layers"][0], xd["k"], xd["v"]
+    shape = r["shape"]
+    o = torch.full_like(q0, 7.0)
+    lse = torch.full((wl.Hq, wl.L), 7.0, device=DEV)
+    idx = torch.full_like(r["idx"], 7)
+    cnt = torch.full_like(r["cnt"], 7)
+    ws = torch.empty(hs2.workspace_bytes(shape) // 4 + 4, device=DEV, dtype=torch.float32)
+    torch.cuda.synchronize()
+    n0 = hs2.hs2_launch_count()
+    hs2.hs2_debug_set(H.WAIT_LIMIT_NS, hs2.DEBUG_FAIL_TMAP)
+    try:
+        calls = [
+            lambda: hs2.hs2_attn_fwd(shape, q0, k, v, None, None, o, lse),
+            lambda: hs2.hs2_full_attn_select(shape, q0, k, v, None, None, o, lse, idx, cnt, ws),
+            lambda: hs2.hs2_sparse_attn(shape, xd["q_layers"][1], k, v, None, None, r["idx"], r["cnt"], o),
+            lambda: hs2.hs2_swa_attn(shape, q0, k, v, 128, o, lse),
+        ]
+        for call in calls:
+            with pytest.raises(hs2.Hs2Error) as e:
+                call()
+            assert e.value.code == hs2.HS2_ERR_CUDA
+    finally:
+        hs2.hs2_debug_set(H.WAIT_LIMIT_NS, 0)
+    torch.cuda.synchronize()
+    assert hs2.hs2_launch_count() == n0
+    assert bool((o == 7.0).all()) and bool((lse == 7.0).all())
+    assert bool((idx == 7).all()) and bool((cnt == 7).all())
+    hs2.hs2_full_attn_select(shape, q0, k, v, None, None, o, lse, idx, cnt, ws)
+    hs2.hs2_sync()
+    assert torch.equal(o, r["o"]) and torch.equal(lse, r["lse"])
+    assert torch.equal(idx, r["idx"]) and torch.equal(cnt, r["cnt"])
+
+
 def test_out_of_range_list_entries_are_reported_not_read():
     """Listed positions outside [0, e_b) are never dereferenced: the gather
     zero-fills them, the softmax masks them, and hs2_sync reports

@@ -21,8 +21,8 @@
 // halves; the halves of both CTAs complete on the leader CTA's full
 // barriers (cta_group::2 TMA).  Warps 2-3 forward "Q ready" to the leader
 // (converting Q to f16 first with an FP8 cache).  In the leader (rank 0) one
-// thread of warp 1 issues every MMA; its commits arrive on the barriers of
-// both CTAs (multicast).  The softmax warps of both CTAs arrive on the
+// thread of warp 1 issues every MMA; each of its commits arrives on the
+// barriers of both CTAs.  The softmax warps of both CTAs arrive on the
 // leader's p_ready barriers.  Every wait is bounded.
 //
 // K/V modes: the bf16 cache, or the layer's f16 copy of an e4m3 cache (K
@@ -105,8 +105,8 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
-// TMA load into this CTA's shared memory completing on a barrier of either
-// CTA of the pair (no multicast).
+// TMA load into this CTA's shared memory (this CTA only) completing on a
+// barrier of either CTA of the pair.
 __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t cluster_bar, int c0,
                                                  int c1, int c2) {
   asm volatile(

@@ -7,6 +7,7 @@
 // word read back by hs2_sync.  No device memory is ever allocated here.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -33,6 +34,21 @@ uint32_t g_flags = 0;
 std::atomic<uint64_t> g_launches{0};
 
 inline int cuda_ok(cudaError_t e) { return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA; }
+
+// NVTX range around each kernel's launch (and each composite call), so that a
+// profiler can attribute and filter launches by name; free when no tool is
+// attached.
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
+
+// Test hook (hs2_debug_set bit 3): every TMA descriptor encoding reports a
+// failure, as a driver error would, so that tests can check that a call
+// fails with HS2_ERR_CUDA before launching anything.
+constexpr uint32_t FLAG_FAIL_TMAP = 8u;
 
 inline int launched() {
   const cudaError_t e = cudaGetLastError();
@@ -100,7 +116,7 @@ EncodeTiledFn encode_fn() {
 int make_map(CUtensorMap* m, const void* base, int L, int H, int64_t tok_stride, int64_t head_stride, int box_h,
              int box_t) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return HS2_ERR_CUDA;
+  if (!enc || (g_flags & FLAG_FAIL_TMAP)) return HS2_ERR_CUDA;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(HD), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(L)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_stride) * 2, static_cast<cuuint64_t>(tok_stride) * 2};
   const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_h), static_cast<cuuint32_t>(box_t)};
@@ -188,6 +204,7 @@ DequantBuf dequant_carve(const hs2_shape* s, uint8_t* base) {
 
 int launch_dequant(const hs2_shape* s, const void* k, const void* v, const float* ks, const float* vs,
                    const DequantBuf& d, cudaStream_t st) {
+  const Range range("hs2 dequant_kv");
   DequantParams p{};
   p.L = s->L;
   p.Hkv = s->Hkv;
@@ -212,6 +229,7 @@ int launch_dequant(const hs2_shape* s, const void* k, const void* v, const float
 // to read the cache itself (bf16 by TMA, or e4m3 converted in the kernel).
 int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void* v, const float* ks,
                     const float* vs, void* o, float* lse, cudaStream_t st, const DequantBuf* dq = nullptr) {
+  const Range range("hs2 attn_fwd (kernel 1)");
   const bool kv8 = s->kv_dtype == HS2_KV_E4M3;
   CUtensorMap mq, mk, mv;
   int rc;
@@ -288,6 +306,7 @@ int launch_attn_fwd(const hs2_shape* s, const void* q, const void* k, const void
 int launch_sparse(const hs2_shape* s, const void* q, const void* k, const void* v, const float* ks,
                   const float* vs, const int32_t* idx, const int32_t* cnt, void* o, cudaStream_t st, int window = 0,
                   float* lse = nullptr) {
+  const Range range(window > 0 ? "hs2 swa_attn (kernel 4, window)" : "hs2 sparse_attn (kernel 4)");
   const int G = s->Hq / s->Hkv;
   const int rows_tok = 128 / G;
   CUtensorMap mq, mk, mv;
@@ -374,6 +393,7 @@ DecodePlan decode_plan(const hs2_shape* s, int n) {
 int launch_decode(const hs2_shape* s, const void* q, const int32_t* positions, int n, const void* k, const void* v,
                   const float* ks, const float* vs, const int32_t* idx, const int32_t* cnt, void* o, void* ws,
                   const DecodePlan& pl, cudaStream_t st) {
+  const Range range("hs2 sparse_decode");
   DecodeParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.q_tok = s->q_tok_stride;
@@ -431,6 +451,7 @@ int launch_importance_g(const CUtensorMap& mq, const CUtensorMap& mk, const ImpP
 int launch_importance(const hs2_shape* s, const void* q, const void* k, const float* ks, const float* lse, int b0,
                       int b1, float* imp, int64_t row_stride, int skip_le, cudaStream_t st,
                       const DequantBuf* dq = nullptr, bool visible = false) {
+  const Range range("hs2 importance (kernel 2)");
   const bool kv8 = s->kv_dtype == HS2_KV_E4M3;
   const int G = s->Hq / s->Hkv;
   const int longest = visible ? std::min(s->L, 64 * b1) : n_cand(s, b1 - 1);
@@ -487,6 +508,7 @@ constexpr uint32_t kBlockSelectSmem = 64u * 1024u;
 
 int launch_select(const hs2_shape* s, const float* imp, int64_t row_stride, int b0, int b1, int32_t* idx,
                   int32_t* cnt, cudaStream_t st, bool blocks = false) {
+  const Range range(blocks ? "hs2 block_select" : "hs2 topk_select (kernel 3)");
   SelParams p{};
   p.L = s->L;
   p.Hkv = s->Hkv;
@@ -778,6 +800,7 @@ int export_rows(const hs2_shape* s, const float* imp, int sb0, int sb1, int64_t 
 int full_attn_select_impl(const hs2_shape* shape, const void* q, const void* k, const void* v, const float* k_scale,
                           const float* v_scale, void* o, float* lse, int32_t* idx, int32_t* cnt, void* workspace,
                           size_t* workspace_bytes, void* stream, bool blocks, const ImpExport& ex) {
+  const Range range(blocks ? "hs2_full_attn_select_blocks" : "hs2_full_attn_select");
   int rc = check_shape(shape);
   if (rc) return rc;
   if (!workspace_bytes) return HS2_ERR_INVALID_ARG;
@@ -870,6 +893,7 @@ int hs2_quantize_kv(int32_t L, int32_t Hkv, const void* src, int64_t src_tok_str
   p.dst_head = dst_head_stride;
   p.scale = scale;
   const int64_t blocks = std::min<int64_t>((static_cast<int64_t>(p.rows) + 63) / 64, 148 * 16);
+  const Range range("hs2 quantize_kv");
   quantize_kv_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
   return launched();
 }

@@ -242,7 +242,7 @@ def hs2_exp2_check(x, y_mufu, y_fma3, y_fma4, stream=None) -> None:
 
 
 # hs2_debug_set flag bits (include/hs2.h)
-DEBUG_SKIP_LOADS, DEBUG_IMP_VISIBLE, DEBUG_FA_CTA_PAIRS = 1, 2, 4
+DEBUG_SKIP_LOADS, DEBUG_IMP_VISIBLE, DEBUG_FA_CTA_PAIRS, DEBUG_FAIL_TMAP = 1, 2, 4, 8
 
 
 def hs2_debug_set(wait_limit_ns: int = 2_000_000_000, flags: int = 0) -> None:
