@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(sp_threads(KV8, WIN), 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->s_full[x], 1);
-      mbar_init(&bars->p_ready[x], 128);
+      mbar_init(&bars->p_ready[x], 4);  // one arrival per softmax warp
       mbar_init(&bars->o_done[x], 1);
       mbar_init(&bars->o_free[x], 128);
       mbar_init(&bars->list_full[x], NLD);
@@ -591,18 +591,18 @@ __global__ void __launch_bounds__(sp_threads(KV8, WIN), 1)
             }
           }
         }
-        // ---- row max: 4 independent chains of 3-input max
-        float mx4[4];
+        // ---- row max: 8 independent chains of 3-input max over 16 values each
+        float mx8[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) mx4[q] = __uint_as_float(sr[q][0]);
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t* v = &sr[q >> 1][(q & 1) * 16];
+          float m = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-#pragma unroll
-          for (int e = 0; e < 15; ++e)
-            mx4[q] = fmax3(mx4[q], __uint_as_float(sr[q][1 + 2 * e]), __uint_as_float(sr[q][2 + 2 * e]));
-          mx4[q] = fmaxf(mx4[q], __uint_as_float(sr[q][31]));
+          for (int e = 0; e < 6; ++e) m = fmax3(m, __uint_as_float(v[3 + 2 * e]), __uint_as_float(v[4 + 2 * e]));
+          mx8[q] = fmaxf(m, __uint_as_float(v[15]));
         }
-        const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
+        const float mx =
+            fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float m_new = fmaxf(m_used, mx * sc);
         float alpha = 1.f;
         const bool resc = m_new > m_used + 8.f;
@@ -636,29 +636,25 @@ __global__ void __launch_bounds__(sp_threads(KV8, WIN), 1)
           f2_unpack(sum2[1], b0, b1);
           l += (a0 + a1) + (b0 + b1);
         }
-        // ---- O rescale (needs P V of the previous tile complete)
-        if (j > 0) {
-          if (!warp_wait(&bars->o_done[x], (t - 1) & 1, p.limit_ns, abort_flag, 332)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, resc)) {
+        // ---- O rescale: P V of the previous tile completed before S of this
+        // one (the MMA thread issues P V(j - 1) first, and s_full's commit
+        // covers every MMA issued before it)
+        if (j > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              uint32_t orr[32];
-              tmem_ld32(o_tm + c * 32, orr);
-              tmem_ld_wait();
-              reg_fence(orr);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(o_tm + c * 32, orr);
+            tmem_ld_wait();
+            reg_fence(orr);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-              tmem_st32(o_tm + c * 32, orr);
-            }
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+            tmem_st32(o_tm + c * 32, orr);
           }
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars->p_ready[x]);
+        __syncwarp();  // one arrival per warp, once all its lanes' stores completed
+        if (lane == 0) mbar_arrive(&bars->p_ready[x]);
       }
       if (!WIN) mbar_arrive(&bars->list_empty[buf]);  // masking is done with this list
       if (!ok) break;
