@@ -1,5 +1,8 @@
 """FP8 KV write (hs2_quantize_kv) against the oracle's quantiser: codes and
-scales bit-exact (both sides divide in fp32 and round to nearest even)."""
+scales bit-exact (the oracle divides in IEEE float32 and rounds to nearest
+even; the kernel reaches the same float32 quotients through a per-row
+reciprocal and two FMA corrections, or the IEEE division for rows of tiny
+amax)."""
 import numpy as np
 import pytest
 import torch
@@ -89,3 +92,34 @@ def test_every_bf16_value_under_many_scales():
     hs2.hs2_sync()
     _check(x, dst, scale)
 
+
+def test_every_scale_mantissa_and_tiny_rows():
+    """Rows whose amax takes each of the 128 bf16 mantissas at three binades
+    (every scale mantissa the kernel can meet), each filled with every bf16
+    value from amax * 2^-20 up to amax of both signs, plus rows of amax below
+    448 * 2^-90 (the kernel's IEEE-division branch) and bf16 subnormals."""
+    rows = []
+    for e in (-3, 4, 12):
+        for m in range(128):
+            a = np.float32((128 + m) / 128 * 2.0 ** e)
+            hi = int(np.array([a], dtype=np.float32).view(np.uint32)[0] >> 16)
+            pats = np.arange(hi - 20 * 128, hi + 1, dtype=np.uint32)
+            vals = (pats << 16).view(np.float32)
+            vals = np.concatenate([vals, -vals[:-1]])
+            n = vals.size // 127 * 127
+            r = vals[:n].reshape(-1, 127)
+            rows.append(np.concatenate([r, np.full((r.shape[0], 1), a, dtype=np.float32)], axis=1))
+    tiny = np.float32(2.0 ** -100)
+    t = (np.arange(1, 128 * 128 + 1, dtype=np.float32) / (128 * 128)).reshape(-1, 128) * tiny
+    t[:, 0] = tiny
+    t[1::2] *= -1
+    rows.append(t.astype(np.float32))
+    sub = (np.arange(1, 129, dtype=np.uint32) << 16).view(np.float32).reshape(1, 128)  # bf16 subnormals
+    rows.append(np.concatenate([sub, -sub]))
+    x = torch.from_numpy(np.concatenate(rows)).to(torch.bfloat16).view(-1, 1, 128)
+    xd = x.to(DEV)
+    dst = torch.empty(x.shape, dtype=torch.uint8, device=DEV)
+    scale = torch.empty(x.shape[:2], device=DEV)
+    hs2.hs2_quantize_kv(xd, dst, scale)
+    hs2.hs2_sync()
+    _check(x, dst, scale)

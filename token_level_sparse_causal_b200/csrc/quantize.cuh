@@ -3,8 +3,8 @@
 //
 // For every (token, KV head) row of 128 bf16 values: amax over the row,
 // scale = amax / 448 in fp32 (1 for an all-zero row), and codes =
-// e4m3(x / scale) with the division in fp32 and saturating round-to-nearest-
-// even conversion.  Grid-stride over rows.  Memory-bound: 256 B read, 128 B +
+// e4m3(x / scale) with the quotient correctly rounded to fp32 (the IEEE
+// quotient) and saturating round-to-nearest-even conversion.  Grid-stride over rows.  Memory-bound: 256 B read, 128 B +
 // 4 B written per row.
 #pragma once
 
@@ -65,8 +65,34 @@ __global__ void __launch_bounds__(256) quantize_kv_kernel(const QuantParams p) {
       for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));  // within the half-warp
       const float scale = (a > 0.f) ? a / 448.0f : 1.0f;
       uint32_t c[4];
+      if (scale >= 0x1p-90f) {
+        // x / scale, correctly rounded, without a division per value:
+        // Markstein's method (P. Markstein, "Computation of elementary
+        // functions on the IBM RISC System/6000 processor", IBM J. Res. Dev.
+        // 34(1), 1990) with y = RN(1 / scale) once per row, q = RN(x y), then
+        // q = RN(q + RN(x - q scale) y) by two FMAs, on value pairs.  Exact
+        // rational arithmetic over every pair of bf16 mantissas of x and of
+        // the row's amax gives RN(x / scale) (tests/test_markstein_division.py;
+        // exponents shift every quantity alike while all stay normal, and the
+        // scale bound keeps the residuals normal for every quotient above
+        // 2^-12, below which both round to a zero code).
+        const float y = __frcp_rn(scale);
+        const uint64_t y2 = f2_pack(y, y), ns2 = f2_pack(-scale, -scale);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) c[q] = e4m3x2_from_f32(v[2 * q] / scale, v[2 * q + 1] / scale);
+        for (int q = 0; q < 4; ++q) {
+          const uint64_t x2 = f2_pack(v[2 * q], v[2 * q + 1]);
+          uint64_t q2 = f2_mul(x2, y2);
+          q2 = f2_fma(f2_fma(q2, ns2, x2), y2, q2);
+          float q0, q1;
+          f2_unpack(q2, q0, q1);
+          // the quotient has x's sign; the correction's RN(+0 + -0) = +0
+          // would lose it for x = -0
+          c[q] = e4m3x2_from_f32(copysignf(q0, v[2 * q]), copysignf(q1, v[2 * q + 1]));
+        }
+      } else {  // rows of amax below 448 * 2^-90: the IEEE division
+#pragma unroll
+        for (int q = 0; q < 4; ++q) c[q] = e4m3x2_from_f32(v[2 * q] / scale, v[2 * q + 1] / scale);
+      }
       if (rowi[k] < p.rows) {
         const int t = rowi[k] / p.Hkv;
         const int hd = rowi[k] - t * p.Hkv;
