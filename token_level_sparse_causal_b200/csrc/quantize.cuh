@@ -4,8 +4,8 @@
 // For every (token, KV head) row of 128 bf16 values: amax over the row,
 // scale = amax / 448 in fp32 (1 for an all-zero row), and codes =
 // e4m3(x / scale) with the quotient correctly rounded to fp32 (the IEEE
-// quotient) and saturating round-to-nearest-even conversion.  Grid-stride over rows.  Memory-bound: 256 B read, 128 B +
-// 4 B written per row.
+// quotient) and saturating round-to-nearest-even conversion.  Grid-stride
+// over rows.  Memory-bound: 256 B read, 128 B + 4 B written per row.
 #pragma once
 
 #include "common.cuh"
