@@ -237,13 +237,15 @@ __device__ void bitonic_sort_smem(uint32_t* a, int np) {
 // as a signed integer are >= those of that float (negative values, -0.0 and
 // negative NaNs are negative integers; positive NaNs lie above +inf in both
 // orders), so one integer compare decides.  Each thread first counts its
-// values (16 in flight), the warp forms a prefix with one shared atomic, and
-// only then do lanes with hits store them.
+// values (16 in flight); a thread with hits reserves that many slots with one
+// shared atomic and stores them.  The slot order is not deterministic, and
+// nothing downstream depends on it (the set is order-free; emission is by
+// position).
 template <bool FAST>
 __device__ __forceinline__ void gather_pass(const float4* row4, int n4, uint32_t tau, uint32_t* ckey,
                                             uint32_t* cpos, uint32_t* count) {
   constexpr int U = 4;  // float4 loads in flight per thread
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
   const int tau_i = static_cast<int>(tau & 0x7FFFFFFFu);
   auto hit = [&](float f, bool live) -> bool {
     return FAST ? (__float_as_int(f) >= tau_i) : (live && order_key(f) >= tau);
@@ -264,18 +266,10 @@ __device__ __forceinline__ void gather_pass(const float4* row4, int n4, uint32_t
     for (int u = 0; u < U; ++u)
       c += (hit(v[u].x, live[u]) ? 1u : 0u) + (hit(v[u].y, live[u]) ? 1u : 0u) + (hit(v[u].z, live[u]) ? 1u : 0u) +
            (hit(v[u].w, live[u]) ? 1u : 0u);
-    uint32_t incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const uint32_t wtot = __shfl_sync(0xffffffffu, incl, 31);
-    if (wtot == 0) continue;  // warp-uniform
-    uint32_t wbase = 0;
-    if (lane == 31) wbase = atomicAdd(count, wtot);
-    uint32_t at = __shfl_sync(0xffffffffu, wbase, 31) + incl - c;
     if (c) {
+      // hits are sparse (about 2k of a row's values pass tau), so the few
+      // lanes with any reserve their slots with one shared atomic each
+      uint32_t at = atomicAdd(count, c);
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const uint32_t p0 = static_cast<uint32_t>(base4 + u * SEL_THREADS + tid) * 4u;
