@@ -86,6 +86,23 @@ struct SpItem {
 };
 
 // The list length of item `it` (0 past the last item).
+// Window mode's item order: CTA c takes it = c, c + grid, ...; this maps
+// each full run of grid * mpairs such indices so that one CTA takes the M-tile
+// pairs of one (block, KV head) back to back, the second finding the window's
+// K/V tiles in L2 right after the first (2.46 -> 2.37 ms at 128k, 64/8 heads,
+// W = 128; the list modes measured 3% slower with it and keep the plain
+// order).  The last, partial run keeps the plain order; the map is a
+// bijection on [0, n_items).
+__device__ __forceinline__ int item_id(const FlashParams& p, int it, int n_items) {
+  if (p.mpairs == 1) return it;
+  const int step = static_cast<int>(gridDim.x);
+  const int run = step * p.mpairs;
+  const int r0 = (it / run) * run;
+  if (r0 + run > n_items) return it;
+  const int l = it - r0;
+  return r0 + (l % step) * p.mpairs + l / step;
+}
+
 __device__ __forceinline__ int item_cnt(const FlashParams& p, int it, int n_items) {
   if (it >= n_items) return 0;
   const int bg = it / p.mpairs;
@@ -96,10 +113,11 @@ __device__ __forceinline__ int item_cnt(const FlashParams& p, int it, int n_item
 // path).  In window mode the keys are the contiguous range the block's
 // windows cover, [max(0, 64 b - W + 1), 64 b + 63], and c is not used.
 template <bool WIN>
-__device__ __forceinline__ SpItem sparse_item(const FlashParams& p, int it, int c) {
+__device__ __forceinline__ SpItem sparse_item(const FlashParams& p, int it, int c, int n_items) {
   SpItem w;
-  w.pair = it % p.mpairs;
-  const int bg = it / p.mpairs;
+  const int id = WIN ? item_id(p, it, n_items) : it;
+  w.pair = id % p.mpairs;
+  const int bg = id / p.mpairs;
   w.g = bg % p.Hkv;
   w.b = bg / p.Hkv;
   w.e_b = min(p.L, 64 * (w.b + 1));
@@ -182,7 +200,7 @@ __global__ void __launch_bounds__(sp_threads(KV8, WIN), 1)
       int c_cur = WIN ? 0 : item_cnt(p, first, n_items), c_nxt = 0;
       for (int it = first; it < n_items; it += step, ++ii, c_cur = c_nxt) {
         c_nxt = WIN ? 0 : item_cnt(p, it + step, n_items);
-        const SpItem w = sparse_item<WIN>(p, it, c_cur);
+        const SpItem w = sparse_item<WIN>(p, it, c_cur, n_items);
         if (w.nt == 0) continue;
         bool ok = true;
         // window mode: key tile j of the item into its ring stage
@@ -233,7 +251,7 @@ __global__ void __launch_bounds__(sp_threads(KV8, WIN), 1)
       int c_cur = WIN ? 0 : item_cnt(p, first, n_items), c_nxt = 0;
       for (int it = first; it < n_items && ok; it += step, c_cur = c_nxt) {
         c_nxt = WIN ? 0 : item_cnt(p, it + step, n_items);
-        const SpItem w = sparse_item<WIN>(p, it, c_cur);
+        const SpItem w = sparse_item<WIN>(p, it, c_cur, n_items);
         const int nt = w.nt;
         if (nt == 0) continue;
         const int nx[2] = {nt, w.nB};
@@ -331,7 +349,7 @@ __global__ void __launch_bounds__(sp_threads(KV8, WIN), 1)
       int c_cur = WIN ? 0 : item_cnt(p, first, n_items), c_nxt = 0;
       for (int it = first; it < n_items && ok; it += step, ++ii, c_cur = c_nxt) {
         c_nxt = WIN ? 0 : item_cnt(p, it + step, n_items);
-        const SpItem w = sparse_item<WIN>(p, it, c_cur);
+        const SpItem w = sparse_item<WIN>(p, it, c_cur, n_items);
         const int buf = ii & 1;
         int32_t* pos_s = pos_base + buf * MAX_LIST;
         // ---- the item's list (the buffer's previous item is done with it)
@@ -525,7 +543,7 @@ __global__ void __launch_bounds__(sp_threads(KV8, WIN), 1)
     int c_cur = WIN ? 0 : item_cnt(p, first, n_items), c_nxt = 0;
     for (int it = first; it < n_items && ok; it += step, ++ii, c_cur = c_nxt) {
       c_nxt = WIN ? 0 : item_cnt(p, it + step, n_items);
-      const SpItem w = sparse_item<WIN>(p, it, c_cur);
+      const SpItem w = sparse_item<WIN>(p, it, c_cur, n_items);
       const int buf = ii & 1;
       const int32_t* pos_s = pos_base + buf * MAX_LIST;
       const int nX = x ? w.nB : w.nt;
